@@ -1,0 +1,518 @@
+"""Benchmark of the sliding-window GQA attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (the headline): single-layer Mistral-7B-shaped chunked prefill, batch
+1, 16384 tokens, W = chunk = 4096, 32 query heads over 8 kv heads, head_dim
+128, bf16 N(0,1) inputs with Q divided by sqrt(128) (scale 1.0).  One step =
+the whole prompt: 4 x (swa_prefill_chunk + swa_cache_append), i.e. slot mapping,
+cache append and chunk attention.  `value` is prompt tokens per second.
+
+Alongside, in the same run and with the same step count:
+  decode   - batch 64 at positions uniform in [4096, 32768), W = 4096 cache per
+             sequence, one swa_decode call per step (tokens/s, HBM GB/s)
+  dense    - the same 16384-token inputs as one causal chunk (W = 16384): the
+             "vanilla attention" side of the pages' 2x SWA claim
+Each reports its kernel's roofline fraction.  Timing: CUDA events on the
+launching stream, L2 flushed (256 MiB write) before every timed step, max over
+ranks.  Under torchrun every rank runs its own replica of the workload (the
+path needs no exchange between GPUs), so `value` is the sum over ranks.
+
+--impl reference times the float64 CPU oracle on the same workload and prints
+the same JSON line (a bounded sample of query rows per step).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from swa_workloads import (DECODE_B64, PREFILL_16K, decode_cache, decode_positions,  # noqa: E402
+                           decode_step_inputs, prefill_inputs)
+
+METRIC = ("prefill tokens/s & TFLOP/s (% bf16 peak); decode tokens/s & HBM GB/s (% peak)")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def prefill_pairs_per_head(L: int, W: int, chunk: int) -> int:
+    """Visible (query, key) pairs of one head over a whole prompt: query i sees
+    min(i + 1, W) keys, however the prompt is chunked."""
+    return sum(min(i + 1, W) for i in range(L))
+
+
+def chunk_pairs_per_head(start: int, T: int, W: int) -> int:
+    return sum(min(start + t + 1, W) for t in range(T))
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while active."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.out.close()
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+        except Exception:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def reduce_max(x: float, world: int) -> float:
+    """Maximum of a per-rank float over all ranks (identity when world == 1)."""
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------
+# our implementation
+# ----------------------------------------------------------------------------
+
+class PrefillRun:
+    """Chunked prefill of one 16384-token prompt through the C ABI."""
+
+    def __init__(self, wl, out_dtype="bf16", device="cuda"):
+        import sliding_window_gqa_chunk_b200 as swa
+        self.swa = swa
+        s = wl.shape
+        self.wl = wl
+        self.L = wl.lengths[0]
+        self.chunk = wl.chunk
+        self.dims = swa.Dims(1, s.n_q_heads, s.n_kv_heads, s.head_dim, s.window, wl.scale,
+                             out_dtype)
+        q, k, v = prefill_inputs(wl, device=device)
+        self.q, self.k, self.v = q, k, v
+        self.out = torch.empty((1, self.L, s.n_q_heads, s.head_dim), dtype=self.dims.torch_out_dtype,
+                               device=device)
+        self.kc, self.vc = swa.new_cache(self.dims, device)
+        n_calls = (self.L + self.chunk - 1) // self.chunk
+        self.starts = [torch.tensor([c * self.chunk], dtype=torch.int32, device=device)
+                       for c in range(n_calls)]
+        self.counts = [torch.tensor([min(self.chunk, self.L - c * self.chunk)], dtype=torch.int32,
+                                    device=device) for c in range(n_calls)]
+        self.n_calls = n_calls
+        # per-chunk views (contiguous: batch 1)
+        self.views = []
+        for c in range(n_calls):
+            a, b = c * self.chunk, min(self.L, (c + 1) * self.chunk)
+            self.views.append(tuple(x[:, a:b] for x in (self.q, self.k, self.v, self.out)))
+        pairs = [chunk_pairs_per_head(c * self.chunk, min(self.chunk, self.L - c * self.chunk),
+                                      s.window) for c in range(n_calls)]
+        self.flops_per_call = [4.0 * s.head_dim * s.n_q_heads * p for p in pairs]
+        self.launches_per_step = 2 * n_calls
+
+    def step(self, events=None):
+        # No cache reset between prompts: chunk 0 (start 0) reads nothing from
+        # the cache, and chunk c > 0 reads only slots chunk c - 1 rewrote.
+        swa = self.swa
+        for c in range(self.n_calls):
+            q, k, v, o = self.views[c]
+            if events is not None:
+                events[c][0].record()
+            swa.prefill_chunk(self.dims, o, q, k, v, self.kc, self.vc, self.starts[c], self.counts[c])
+            if events is not None:
+                events[c][1].record()
+            swa.cache_append(self.dims, self.kc, self.vc, k, v, self.starts[c], self.counts[c])
+
+
+def run_prefill_e2e(run: PrefillRun, steps: int, warmup: int, flush):
+    """Same workload through the public API with pinned host buffers: every step
+    copies q/k/v host->device, runs the 4 chunks, and copies out device->host."""
+    qh = run.q.cpu().pin_memory()
+    kh = run.k.cpu().pin_memory()
+    vh = run.v.cpu().pin_memory()
+    oh = torch.empty(run.out.shape, dtype=run.out.dtype).pin_memory()
+    times = []
+    for i in range(warmup + steps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        run.q.copy_(qh, non_blocking=True)
+        run.k.copy_(kh, non_blocking=True)
+        run.v.copy_(vh, non_blocking=True)
+        run.step()
+        oh.copy_(run.out, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= warmup:
+            times.append(e0.elapsed_time(e1))
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size()
+    return sum(times) / len(times), h2d, d2h
+
+
+class DecodeRun:
+    """One decode step of batch 64 (positions uniform in [4096, 32768))."""
+
+    def __init__(self, wl, out_dtype="bf16", device="cuda"):
+        import sliding_window_gqa_chunk_b200 as swa
+        self.swa = swa
+        s = wl.shape
+        self.wl = wl
+        self.dims = swa.Dims(wl.batch, s.n_q_heads, s.n_kv_heads, s.head_dim, s.window, wl.scale,
+                             out_dtype)
+        self.kc, self.vc = decode_cache(wl, 0, device=device)
+        self.pos0 = decode_positions(wl, device=device)
+        self.pos = self.pos0.clone()
+        self.inputs = [decode_step_inputs(wl, i, 0, device=device) for i in range(4)]
+        self.out = torch.empty((wl.batch, s.n_q_heads, s.head_dim), dtype=self.dims.torch_out_dtype,
+                               device=device)
+        self.ws = torch.empty(swa.decode_workspace_size(self.dims), dtype=torch.uint8, device=device)
+        self.i = 0
+        B, W, Hkv, d, Hq = wl.batch, s.window, s.n_kv_heads, s.head_dim, s.n_q_heads
+        out_b = 4 if out_dtype == "f32" else 2
+        # algorithmic bytes per step: the W cached keys+values of every (seq, kv head),
+        # q, the new k/v (read once, written once into the cache), the output
+        self.bytes_per_step = B * (2 * W * Hkv * d * 2 + Hq * d * 2 + 2 * Hkv * d * 2 * 2 +
+                                   Hq * d * out_b)
+        self.launches_per_step = 1 if swa.decode_workspace_size(self.dims) <= 16 else 2
+
+    def step(self, events=None):
+        q, k, v = self.inputs[self.i % len(self.inputs)]
+        self.i += 1
+        if events is not None:
+            events[0].record()
+        self.swa.decode(self.dims, self.out, q, k, v, self.kc, self.vc, self.pos, self.ws)
+        if events is not None:
+            events[1].record()
+        self.pos.add_(1)
+
+
+def time_steps(fn, steps, warmup, flush, n_events=1):
+    """Per-step CUDA-event timing with an L2 flush before every step (outside the
+    timed interval).  Returns (mean step ms, mean per-event-pair ms list)."""
+    for _ in range(warmup):
+        flush()
+        fn(None)
+    torch.cuda.synchronize()
+    step_ms, pair_ms = [], [[] for _ in range(n_events)]
+    for _ in range(steps):
+        flush()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n_events)]
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        fn(ev)
+        s1.record()
+        torch.cuda.synchronize()
+        step_ms.append(s0.elapsed_time(s1))
+        for i, (a, b) in enumerate(ev):
+            pair_ms[i].append(a.elapsed_time(b))
+    return (sum(step_ms) / len(step_ms),
+            [sum(x) / len(x) for x in pair_ms])
+
+
+def bench_ours(args, world, rank, local):
+    import sliding_window_gqa_chunk_b200 as swa
+    from sliding_window_gqa_chunk_b200.csrc import build as swa_build
+    swa_build.build()
+    swa.load_library()
+    dev = f"cuda:{local}"
+    peaks = load_peaks()
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.fill_(1)
+
+    wl = PREFILL_16K
+    run = PrefillRun(wl, "bf16", dev)
+    step = lambda ev: run.step(ev)  # noqa: E731
+
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ms, per_call = time_steps(step, args.steps, args.warmup, flush, n_events=run.n_calls)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = clk.summary()
+    ms_max = reduce_max(ms, world)
+    swa.device_status()
+
+    tokens = run.L
+    value = world * tokens / (ms_max / 1e3)
+    flops_step = sum(run.flops_per_call)
+    kernel_ms = sum(per_call)                   # prefill kernel time per step
+    avg_launch_ms = kernel_ms / run.n_calls
+    avg_flops = flops_step / run.n_calls
+    achieved_tflops = avg_flops / (avg_launch_ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops"]
+
+    # decode phase
+    dec = DecodeRun(DECODE_B64, "bf16", dev)
+    dms, dpair = time_steps(lambda ev: dec.step(ev), args.steps, args.warmup, flush, n_events=1)
+    dms_max = reduce_max(dms, world)
+    dec_kernel_ms = dpair[0]
+    dec_gbs = dec.bytes_per_step / (dec_kernel_ms / 1e3) / 1e9
+    swa.device_status()
+
+    # dense causal comparator on the same inputs
+    dense_dims = swa.Dims(1, 32, 8, 128, 16384, wl.scale, "bf16")
+    dkc, dvc = swa.new_cache(dense_dims, dev)
+    zero = torch.zeros(1, dtype=torch.int32, device=dev)
+    full = torch.tensor([16384], dtype=torch.int32, device=dev)
+
+    def dense_step(ev):
+        if ev is not None:
+            ev[0][0].record()
+        swa.prefill_chunk(dense_dims, run.out, run.q, run.k, run.v, dkc, dvc, zero, full)
+        if ev is not None:
+            ev[0][1].record()
+
+    dense_ms, dense_pair = time_steps(dense_step, max(2, args.steps // 2), 2, flush, n_events=1)
+    dense_flops = 4.0 * 128 * 32 * prefill_pairs_per_head(16384, 16384, 16384)
+    swa.device_status()
+
+    # end to end through the public API with host buffers
+    e2e_ms, h2d, d2h = run_prefill_e2e(run, args.steps, min(args.warmup, 3), flush)
+    e2e_ms = reduce_max(e2e_ms, world)
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_max, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "batch": 1, "seq_len": run.L, "window": wl.shape.window,
+                   "chunk": wl.chunk, "n_q_heads": 32, "n_kv_heads": 8, "head_dim": 128,
+                   "out_dtype": "bf16", "l2": "flushed (256 MiB write) before every timed step",
+                   "parallelism": f"replicas x{world}"},
+        "tflops": round(flops_step / (ms_max / 1e3) / 1e12, 1),
+        "roofline": {"kernel": "swa_prefill_kernel", "bound": "tensor",
+                     "achieved": round(achieved_tflops, 1), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved_tflops / peak, 4),
+                     "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+                     "algorithmic_flops_per_launch": avg_flops, "traffic": None},
+        "decode": {"workload": DECODE_B64.name, "batch": DECODE_B64.batch,
+                   "tokens_per_s": round(world * DECODE_B64.batch / (dms_max / 1e3), 1),
+                   "ms_per_step": round(dms_max, 4),
+                   "roofline": {"kernel": "swa_decode_kernel+combine", "bound": "hbm",
+                                "achieved": round(dec_gbs, 1), "peak": peaks["hbm_gbs"],
+                                "unit": "GB/s", "frac": round(dec_gbs / peaks["hbm_gbs"], 4),
+                                "peak_source": f"{peaks['source']} hbm_gbs",
+                                "algorithmic_bytes_per_launch": dec.bytes_per_step,
+                                "traffic": None},
+                   "gpu_launches_per_step": dec.launches_per_step},
+        "dense": {"workload": "dense_causal_16k", "ms": round(dense_pair[0], 4),
+                  "tflops": round(dense_flops / (dense_pair[0] / 1e3) / 1e12, 1),
+                  "swa_speedup_vs_dense": round(dense_pair[0] / kernel_ms, 3)},
+        "e2e": {"value": round(world * tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": run.launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
+    return line
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle (reference arm and cpu_baseline)
+# ----------------------------------------------------------------------------
+
+def oracle_sample(wl, rows: int, q, k, v):
+    """The oracle on `rows` query tokens of the last chunk (all heads), each
+    attending to its full window: returns seconds."""
+    import numpy as np
+    import oracle
+    L, W = wl.lengths[0], wl.shape.window
+    st = L - wl.chunk                      # last chunk: every row sees W keys
+    lo = st - W + 1
+    qs = q[0, st:st + rows]
+    ks = k[0, max(0, lo):st + rows]
+    vs = v[0, max(0, lo):st + rows]
+    t0 = time.perf_counter()
+    oracle.attend(qs, np.arange(st, st + rows), ks, vs, np.arange(max(0, lo), st + rows), W,
+                  wl.scale)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(wl, budget_s=12.0):
+    import oracle
+    q, k, v = prefill_inputs(wl, device="cpu")
+    rows, spent, total_rows = 64, 0.0, 0
+    while spent < budget_s and total_rows + rows <= wl.chunk:
+        spent += oracle_sample(wl, rows, q, k, v)
+        total_rows += rows
+        rows = min(rows * 2, 512)
+    return {"value": round(total_rows / spent, 2), "unit": "tokens/s", "cores": oracle.max_threads(),
+            "kind": "oracle",
+            "sample": f"{total_rows} query tokens of the last 4096-token chunk (all 32 heads, "
+                      f"4096 keys each), float64 C oracle, OpenMP"}
+
+
+def bench_reference(args, world, rank):
+    if rank != 0:
+        return None
+    import oracle
+    oracle.build()
+    wl = PREFILL_16K
+    q, k, v = prefill_inputs(wl, device="cpu")
+    rows = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample(wl, rows, q, k, v)
+    times = [oracle_sample(wl, rows, q, k, v) for _ in range(args.steps)]
+    per = sum(times) / len(times)
+    value = rows / per
+    sample = (f"{rows} query tokens of the last 4096-token chunk per step (all 32 heads, 4096 "
+              f"keys each), float64 C oracle, OpenMP")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(per * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": 1, "seq_len": wl.lengths[0],
+                   "window": wl.shape.window, "chunk": wl.chunk, "n_q_heads": 32,
+                   "n_kv_heads": 8, "head_dim": 128, "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s",
+                         "cores": oracle.max_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--ref-rows", type=int, default=128)
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        # CPU oracle only: no process group; under torchrun rank 0 alone works.
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        line = bench_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            line = bench_reference(args, world, rank)
+        else:
+            line = bench_ours(args, world, rank, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

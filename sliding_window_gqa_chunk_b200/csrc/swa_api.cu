@@ -1,0 +1,335 @@
+// swa_api.cu - the extern "C" entry points of libswa.so (declared in swa.h):
+// argument validation, the thread-local error message, the per-device status
+// word, TMA descriptor encoding for the prefill, and kernel dispatch.
+//
+// Nothing here allocates device memory.  Every check that can be made on the
+// host is made before the first launch, so a call that returns an argument
+// error has enqueued nothing.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <initializer_list>
+#include <mutex>
+
+#include "swa.h"
+#include "swa_internal.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int ok() {
+  g_last_error[0] = '\0';
+  return SWA_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(SWA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- status word
+// One int per device, written by kernels with atomicCAS (first error wins).
+__device__ int g_swa_status;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_status_mu;
+int* g_status_ptr[kMaxDevices] = {};
+
+// Device address of g_swa_status on the current device (looked up once per device).
+int status_ptr(int** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(SWA_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  if (g_status_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_swa_status);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  *out = g_status_ptr[dev];
+  return SWA_OK;
+}
+
+// ---------------------------------------------------------------- validation
+int check_dims(const swa_dims* d) {
+  if (d == nullptr) return fail(SWA_ERR_INVALID_ARG, "dims is NULL");
+  if (d->batch < 1 || d->batch > 65535) return fail(SWA_ERR_INVALID_ARG, "batch %d not in [1, 65535]", d->batch);
+  if (d->n_q_heads < 1 || d->n_kv_heads < 1)
+    return fail(SWA_ERR_INVALID_ARG, "head counts must be >= 1 (Hq=%d, Hkv=%d)", d->n_q_heads, d->n_kv_heads);
+  if (d->n_q_heads % d->n_kv_heads != 0)
+    return fail(SWA_ERR_UNSUPPORTED, "Hq=%d is not a multiple of Hkv=%d", d->n_q_heads, d->n_kv_heads);
+  if (d->n_q_heads / d->n_kv_heads > 16)
+    return fail(SWA_ERR_UNSUPPORTED, "group size Hq/Hkv=%d above 16", d->n_q_heads / d->n_kv_heads);
+  if (d->n_kv_heads > 65535 || d->n_q_heads > 65535)
+    return fail(SWA_ERR_INVALID_ARG, "head count above 65535");
+  if (d->head_dim != 16 && d->head_dim != 64 && d->head_dim != 128)
+    return fail(SWA_ERR_UNSUPPORTED, "head_dim %d not in {16, 64, 128}", d->head_dim);
+  if (d->window < 1) return fail(SWA_ERR_INVALID_ARG, "window %d < 1", d->window);
+  if (!(d->scale > 0.f) || !std::isfinite(d->scale))
+    return fail(SWA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (d->out_dtype != SWA_DTYPE_BF16 && d->out_dtype != SWA_DTYPE_F32)
+    return fail(SWA_ERR_INVALID_ARG, "out_dtype %d unknown", d->out_dtype);
+  return SWA_OK;
+}
+
+int check_ptrs(const char* names, std::initializer_list<const void*> ptrs) {
+  int i = 0;
+  for (const void* p : ptrs) {
+    if (p == nullptr) return fail(SWA_ERR_INVALID_ARG, "pointer #%d of (%s) is NULL", i, names);
+    if (!aligned16(p)) return fail(SWA_ERR_INVALID_ARG, "pointer #%d of (%s) is not 16-byte aligned", i, names);
+    ++i;
+  }
+  return SWA_OK;
+}
+
+int check_int_ptrs(const char* names, std::initializer_list<const int32_t*> ptrs) {
+  int i = 0;
+  for (const int32_t* p : ptrs) {
+    if (p == nullptr) return fail(SWA_ERR_INVALID_ARG, "pointer #%d of (%s) is NULL", i, names);
+    if ((reinterpret_cast<uintptr_t>(p) & 3u) != 0)
+      return fail(SWA_ERR_INVALID_ARG, "pointer #%d of (%s) is not 4-byte aligned", i, names);
+    ++i;
+  }
+  return SWA_OK;
+}
+
+// ---------------------------------------------------------------- TMA encoding
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+int get_encode(EncodeTiledFn* fn) {
+  static EncodeTiledFn cached = nullptr;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lk(mu);
+  if (cached == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || p == nullptr)
+      return fail(SWA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found (%s)", cudaGetErrorName(e));
+    cached = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  *fn = cached;
+  return SWA_OK;
+}
+
+// rank-`rank` bf16 map, dims innermost first, byte strides of dims 1..rank-1.
+int encode_map(EncodeTiledFn fn, CUtensorMap* map, const void* ptr, int rank, const cuuint64_t* dims,
+               const cuuint64_t* strides, const cuuint32_t* box, int swizzle_bytes, const char* what) {
+  cuuint32_t estride[5] = {1, 1, 1, 1, 1};
+  CUtensorMapSwizzle swz = swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                           : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                           : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                 : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(ptr), dims,
+                  strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SWA_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed with CUresult %d", what, (int)r);
+  return SWA_OK;
+}
+
+}  // namespace
+
+namespace swa {
+
+DecodeSplit decode_split(int batch, int n_kv_heads, int window) {
+  // Aim for about four resident 128-thread CTAs per SM on a 148-SM B200; each
+  // split is a multiple of 64 slots (16 per warp).
+  const long long units = (long long)batch * n_kv_heads;
+  const long long target = 148LL * 4;
+  long long splits = (target + units - 1) / units;
+  const long long max_splits = (window + 63) / 64;
+  if (splits > max_splits) splits = max_splits;
+  if (splits < 1) splits = 1;
+  long long per = (window + splits - 1) / splits;
+  per = (per + 63) / 64 * 64;
+  DecodeSplit s;
+  s.slots_per_split = (int)per;
+  s.n_splits = (int)((window + per - 1) / per);
+  return s;
+}
+
+}  // namespace swa
+
+extern "C" {
+
+int swa_abi_version(void) { return 100; }
+
+const char* swa_last_error(void) { return g_last_error; }
+
+int swa_cache_append(const swa_dims* dims, void* k_cache, void* v_cache, const void* k, const void* v,
+                     int32_t max_tokens, const int32_t* start_pos, const int32_t* n_tokens, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_ptrs("k_cache, v_cache, k, v", {k_cache, v_cache, k, v}))) return rc;
+  if ((rc = check_int_ptrs("start_pos, n_tokens", {start_pos, n_tokens}))) return rc;
+  if (max_tokens < 1 || max_tokens > dims->window)
+    return fail(SWA_ERR_INVALID_ARG, "max_tokens %d not in [1, window=%d]", max_tokens, dims->window);
+  int* status = nullptr;
+  if ((rc = status_ptr(&status))) return rc;
+  swa::AppendParams p;
+  p.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  p.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.start_pos = start_pos;
+  p.n_tokens = n_tokens;
+  p.status = status;
+  p.batch = dims->batch;
+  p.n_kv_heads = dims->n_kv_heads;
+  p.head_dim = dims->head_dim;
+  p.window = dims->window;
+  p.max_tokens = max_tokens;
+  cudaError_t e = swa::launch_append(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "swa_cache_append launch");
+  return ok();
+}
+
+int swa_prefill_chunk(const swa_dims* dims, void* out, const void* q, const void* k, const void* v,
+                      int32_t max_tokens, const void* k_cache, const void* v_cache, const int32_t* start_pos,
+                      const int32_t* n_tokens, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_ptrs("out, q, k, v, k_cache, v_cache", {out, q, k, v, k_cache, v_cache}))) return rc;
+  if ((rc = check_int_ptrs("start_pos, n_tokens", {start_pos, n_tokens}))) return rc;
+  if (max_tokens < 1 || max_tokens > dims->window)
+    return fail(SWA_ERR_INVALID_ARG, "max_tokens %d not in [1, window=%d]", max_tokens, dims->window);
+  const int B = dims->batch, Hq = dims->n_q_heads, Hkv = dims->n_kv_heads, D = dims->head_dim;
+  const int W = dims->window;
+  int* status = nullptr;
+  if ((rc = status_ptr(&status))) return rc;
+  EncodeTiledFn enc = nullptr;
+  if ((rc = get_encode(&enc))) return rc;
+
+  int box_d = 0, swz = 0;
+  swa::prefill_map_geometry(D, &box_d, &swz);
+  swa::PrefillMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  const cuuint64_t es = 2;  // bf16
+  {
+    cuuint64_t dims4[4] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)max_tokens, (cuuint64_t)B};
+    cuuint64_t str4[3] = {D * es, (cuuint64_t)Hq * D * es, (cuuint64_t)max_tokens * Hq * D * es};
+    cuuint32_t box4[4] = {(cuuint32_t)box_d, 1, 128, 1};
+    if ((rc = encode_map(enc, &maps.q, q, 4, dims4, str4, box4, swz, "q"))) return rc;
+  }
+  {
+    cuuint64_t dims4[4] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)max_tokens, (cuuint64_t)B};
+    cuuint64_t str4[3] = {D * es, (cuuint64_t)Hkv * D * es, (cuuint64_t)max_tokens * Hkv * D * es};
+    cuuint32_t box4[4] = {(cuuint32_t)box_d, 1, 128, 1};
+    if ((rc = encode_map(enc, &maps.k, k, 4, dims4, str4, box4, swz, "k"))) return rc;
+    if ((rc = encode_map(enc, &maps.v, v, 4, dims4, str4, box4, swz, "v"))) return rc;
+  }
+  {
+    cuuint64_t dims3[3] = {(cuuint64_t)D, (cuuint64_t)W, (cuuint64_t)B * Hkv};
+    cuuint64_t str3[2] = {D * es, (cuuint64_t)W * D * es};
+    cuuint32_t box3[3] = {(cuuint32_t)box_d, 128, 1};
+    if ((rc = encode_map(enc, &maps.kc, k_cache, 3, dims3, str3, box3, swz, "k_cache"))) return rc;
+    if ((rc = encode_map(enc, &maps.vc, v_cache, 3, dims3, str3, box3, swz, "v_cache"))) return rc;
+  }
+
+  swa::PrefillParams p;
+  p.out = out;
+  p.start_pos = start_pos;
+  p.n_tokens = n_tokens;
+  p.status = status;
+  p.batch = B;
+  p.n_q_heads = Hq;
+  p.n_kv_heads = Hkv;
+  p.head_dim = D;
+  p.window = W;
+  p.max_tokens = max_tokens;
+  p.heads_per_cta = ((Hq / Hkv) % 2 == 0) ? 2 : 1;
+  p.n_q_tiles = (max_tokens + 127) / 128;
+  p.scale_log2 = dims->scale * 1.4426950408889634f;
+  p.out_f32 = dims->out_dtype == SWA_DTYPE_F32;
+  cudaError_t e = swa::launch_prefill(p, maps, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "swa_prefill_chunk launch");
+  return ok();
+}
+
+size_t swa_decode_workspace_size(const swa_dims* dims) {
+  if (check_dims(dims) != SWA_OK) return 0;
+  const swa::DecodeSplit sp = swa::decode_split(dims->batch, dims->n_kv_heads, dims->window);
+  if (sp.n_splits <= 1) return 16;  // nothing needed; a non-zero size keeps callers simple
+  const size_t bh = (size_t)dims->batch * dims->n_q_heads * sp.n_splits;
+  return bh * dims->head_dim * sizeof(float) + bh * 2 * sizeof(float);
+}
+
+int swa_decode(const swa_dims* dims, void* out, const void* q, const void* k_new, const void* v_new,
+               void* k_cache, void* v_cache, const int32_t* pos, void* workspace, size_t workspace_bytes,
+               void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_ptrs("out, q, k_new, v_new, k_cache, v_cache, workspace",
+                       {out, q, k_new, v_new, k_cache, v_cache, workspace})))
+    return rc;
+  if ((rc = check_int_ptrs("pos", {pos}))) return rc;
+  const size_t need = swa_decode_workspace_size(dims);
+  if (workspace_bytes < need)
+    return fail(SWA_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
+  int* status = nullptr;
+  if ((rc = status_ptr(&status))) return rc;
+  const swa::DecodeSplit sp = swa::decode_split(dims->batch, dims->n_kv_heads, dims->window);
+  swa::DecodeParams p;
+  p.out = out;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
+  p.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
+  p.k_cache_w = static_cast<__nv_bfloat16*>(k_cache);
+  p.v_cache_w = static_cast<__nv_bfloat16*>(v_cache);
+  p.pos = pos;
+  const size_t bh = (size_t)dims->batch * dims->n_q_heads * sp.n_splits;
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_ml = static_cast<float*>(workspace) + bh * dims->head_dim;
+  p.status = status;
+  p.batch = dims->batch;
+  p.n_q_heads = dims->n_q_heads;
+  p.n_kv_heads = dims->n_kv_heads;
+  p.head_dim = dims->head_dim;
+  p.window = dims->window;
+  p.n_splits = sp.n_splits;
+  p.slots_per_split = sp.slots_per_split;
+  p.scale_log2 = dims->scale * 1.4426950408889634f;
+  p.out_f32 = dims->out_dtype == SWA_DTYPE_F32;
+  cudaError_t e = swa::launch_decode(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "swa_decode launch");
+  return ok();
+}
+
+int swa_device_status(void* stream) {
+  int* status = nullptr;
+  int rc = status_ptr(&status);
+  if (rc) return rc;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int value = 0;
+  e = cudaMemcpy(&value, status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
+  const int zero = 0;
+  e = cudaMemcpy(status, &zero, sizeof(int), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
+  if (value != SWA_OK) return fail(value, "device status %d raised by a kernel", value);
+  return ok();
+}
+
+}  // extern "C"

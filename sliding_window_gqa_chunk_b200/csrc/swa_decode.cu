@@ -1,0 +1,407 @@
+// swa_decode.cu - single-token decode over the rolling cache (Mistral 7B,
+// section 2, Rolling Buffer Cache paragraph; token-by-token generation in the
+// Pre-fill and Chunking paragraph).
+//
+// At position pos the new key/value go to slot pos mod W and the query attends
+// over the min(pos + 1, W) cached positions (pos - W, pos].  The cache is the
+// HBM-bound part: every (sequence, kv head) streams W slots x d x 2 B of keys
+// and the same of values, and does ~2 x G x d FMAs per slot.  So one warp
+// handles all G query heads of its kv head (the GQA group shares each load),
+// and the dot products run on the tensor cores through mma.sync m16n8k16 so
+// the CUDA cores only do the online softmax:
+//
+//   S^T[slot][head] = K[slot][:] . Q[head][:]    (M = 16 slots, N = 8 heads, K = d)
+//   O^T[d][head]   += V^T[d][slot] . P^T[slot][head]  (M = 16 d, N = 8 heads, K = 16 slots)
+//
+// Fragments come straight from global memory with 16-byte loads, no shared
+// memory: a dot product over d is invariant under any permutation of d applied
+// to both K and Q, so each lane loads contiguous 16-byte pieces and the d index
+// is relabelled to match the mma fragment layout; the PV product uses a second
+// relabelling of d (undone when O is stored) and pairs consecutive slots with
+// byte permutes.  P^T goes from the S accumulator layout to the B-operand
+// layout with one movmatrix.trans per 8x8 block.
+//
+// Work split: grid (n_splits, Hkv, B); a CTA of 4 warps covers one split of
+// the W slots; warps take interleaved 16-slot blocks, merge their (m, l, O)
+// in shared memory, and write either the final output (one split) or an fp32
+// partial for swa_decode_combine_kernel.  The CTA whose split holds slot
+// pos mod W writes the new key/value there; every lane that would read that
+// slot reads k_new / v_new instead, so no CTA ever reads a slot that is being
+// written.
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "swa_common.cuh"
+#include "swa_internal.h"
+
+namespace swa {
+
+namespace {
+
+constexpr int kDecodeWarps = 4;
+constexpr int kBlockSlots = 16;
+
+// Physical element offset (within a row) of lane-quad t's key piece `j`
+// (K rows and Q rows use the same relabelling of d).
+template <int D>
+__device__ __forceinline__ int k_piece_offset(int t, int j) {
+  if constexpr (D == 16) {
+    return t * 4;
+  } else {
+    return j * 32 + t * 8;
+  }
+}
+
+// Physical element offset of lane-group g's value piece `c` (PV relabelling).
+template <int D>
+__device__ __forceinline__ int v_piece_offset(int g, int c) {
+  if constexpr (D == 16) {
+    return g * 2;
+  } else {
+    return c * 64 + g * 8;
+  }
+}
+
+template <int D>
+struct Frag {
+  // words of one K row held by a lane: D/4 bf16 -> D/8 words
+  static constexpr int kKWords = D / 8;
+  // words of one V row held by a lane: D/8 bf16 -> D/16 words
+  static constexpr int kVWords = D / 16;
+  static constexpr int kKSteps = D / 16;   // mma k-steps of the QK product
+  static constexpr int kMTiles = D / 16;   // m-tiles of the PV product
+};
+
+// Loads the words of one row (key: kKWords, value: kVWords) into regs.
+template <int D>
+__device__ __forceinline__ void load_k_row(uint32_t (&w)[Frag<D>::kKWords], const __nv_bfloat16* row,
+                                           int t, bool valid) {
+  if constexpr (D == 16) {
+    uint2 x = valid ? ldg_stream8(row + k_piece_offset<D>(t, 0)) : make_uint2(0, 0);
+    w[0] = x.x;
+    w[1] = x.y;
+  } else {
+#pragma unroll
+    for (int j = 0; j < D / 32; ++j) {
+      uint4 x = valid ? ldg_stream(row + k_piece_offset<D>(t, j)) : make_uint4(0, 0, 0, 0);
+      w[4 * j + 0] = x.x;
+      w[4 * j + 1] = x.y;
+      w[4 * j + 2] = x.z;
+      w[4 * j + 3] = x.w;
+    }
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void load_v_row(uint32_t (&w)[Frag<D>::kVWords], const __nv_bfloat16* row,
+                                           int g, bool valid) {
+  if constexpr (D == 16) {
+    w[0] = valid ? ldg_stream4(row + v_piece_offset<D>(g, 0)) : 0u;
+  } else {
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      uint4 x = valid ? ldg_stream(row + v_piece_offset<D>(g, c)) : make_uint4(0, 0, 0, 0);
+      w[4 * c + 0] = x.x;
+      w[4 * c + 1] = x.y;
+      w[4 * c + 2] = x.z;
+      w[4 * c + 3] = x.w;
+    }
+  }
+}
+
+template <typename OutT>
+__device__ __forceinline__ void store_out(OutT* dst, float x);
+template <>
+__device__ __forceinline__ void store_out<float>(float* dst, float x) { *dst = x; }
+template <>
+__device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* dst, float x) {
+  *dst = __float2bfloat16_rn(x);
+}
+
+}  // namespace
+
+// NT = number of 8-head n-tiles (ceil(G / 8)).
+template <int D, int NT, typename OutT>
+__global__ void __launch_bounds__(kDecodeWarps * 32)
+swa_decode_kernel(const DecodeParams p) {
+  using F = Frag<D>;
+  extern __shared__ float smem[];
+
+  const int split = blockIdx.x;
+  const int kvh = blockIdx.y;
+  const int b = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2;
+  const int t = lane & 3;
+  const int G = p.n_q_heads / p.n_kv_heads;
+  const int W = p.window;
+
+  const long long pos = p.pos[b];
+  if (pos < 0) {
+    if (threadIdx.x == 0) raise_status(p.status, SWA_ERR_DEVICE_ARG);
+    return;
+  }
+  const int n_valid = (int)(pos + 1 < (long long)W ? pos + 1 : (long long)W);
+  const int s_new = (int)(pos % W);
+  const int r_begin = split * p.slots_per_split;
+  const int r_stop = r_begin + p.slots_per_split;
+  const int r_end = r_stop < n_valid ? r_stop : n_valid;
+
+  const size_t head_stride = (size_t)W * D;
+  const __nv_bfloat16* kc = p.k_cache + ((size_t)b * p.n_kv_heads + kvh) * head_stride;
+  const __nv_bfloat16* vc = p.v_cache + ((size_t)b * p.n_kv_heads + kvh) * head_stride;
+  const __nv_bfloat16* kn = p.k_new + ((size_t)b * p.n_kv_heads + kvh) * D;
+  const __nv_bfloat16* vn = p.v_new + ((size_t)b * p.n_kv_heads + kvh) * D;
+
+  // The split owning slot pos mod W stores the new key/value there.  No lane of
+  // any CTA reads that slot from the cache (they read k_new / v_new).
+  if (warp == 0 && s_new >= r_begin && s_new < r_stop) {
+    for (int i = lane; i < D / 8; i += 32) {
+      reinterpret_cast<uint4*>(p.k_cache_w + ((size_t)b * p.n_kv_heads + kvh) * head_stride +
+                               (size_t)s_new * D)[i] = reinterpret_cast<const uint4*>(kn)[i];
+      reinterpret_cast<uint4*>(p.v_cache_w + ((size_t)b * p.n_kv_heads + kvh) * head_stride +
+                               (size_t)s_new * D)[i] = reinterpret_cast<const uint4*>(vn)[i];
+    }
+  }
+
+  // Q as the B operand of S^T = K Q^T: lane (g, t) holds head 8*nt + g.
+  uint32_t qf[NT][F::kKWords];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int hl = nt * 8 + g;
+    const bool hv = hl < G;
+    const __nv_bfloat16* qrow = p.q + ((size_t)b * p.n_q_heads + (size_t)kvh * G + (hv ? hl : 0)) * D;
+    load_k_row<D>(qf[nt], qrow, t, hv);
+  }
+
+  float o[NT][F::kMTiles][4];
+  float m_run[NT][2];
+  float l_run[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int mt = 0; mt < F::kMTiles; ++mt) {
+      o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
+    }
+    m_run[nt][0] = m_run[nt][1] = -CUDART_INF_F;
+    l_run[nt][0] = l_run[nt][1] = 0.f;
+  }
+  const float sl2 = p.scale_log2;
+
+  for (int blk = r_begin + warp * kBlockSlots; blk < r_end; blk += kDecodeWarps * kBlockSlots) {
+    // ---- loads: K rows blk+g, blk+8+g; V rows blk+2t, +1, +8, +9 ----
+    uint32_t kw0[F::kKWords], kw1[F::kKWords];
+    {
+      const int r0 = blk + g, r1 = blk + 8 + g;
+      load_k_row<D>(kw0, r0 == s_new ? kn : kc + (size_t)r0 * D, t, r0 < r_end);
+      load_k_row<D>(kw1, r1 == s_new ? kn : kc + (size_t)r1 * D, t, r1 < r_end);
+    }
+    uint32_t vw[4][F::kVWords];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = blk + 2 * t + (i & 1) + (i >> 1) * 8;
+      load_v_row<D>(vw[i], r == s_new ? vn : vc + (size_t)r * D, g, r < r_end);
+    }
+    const bool ok0 = blk + g < r_end;
+    const bool ok1 = blk + 8 + g < r_end;
+
+    uint32_t pb[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < F::kKSteps; ++ks) {
+        // k-step ks uses words 2*ks and 2*ks+1 of each row's piece list
+        mma_16816(s, kw0[2 * ks], kw1[2 * ks], kw0[2 * ks + 1], kw1[2 * ks + 1],
+                  qf[nt][2 * ks], qf[nt][2 * ks + 1]);
+      }
+      // s[0]: (slot g, head 2t)   s[1]: (slot g, head 2t+1)
+      // s[2]: (slot g+8, head 2t) s[3]: (slot g+8, head 2t+1)
+      s[0] = ok0 ? s[0] * sl2 : -CUDART_INF_F;
+      s[1] = ok0 ? s[1] * sl2 : -CUDART_INF_F;
+      s[2] = ok1 ? s[2] * sl2 : -CUDART_INF_F;
+      s[3] = ok1 ? s[3] * sl2 : -CUDART_INF_F;
+      float mx0 = fmaxf(s[0], s[2]);
+      float mx1 = fmaxf(s[1], s[3]);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+      }
+      const float mn0 = fmaxf(m_run[nt][0], mx0);
+      const float mn1 = fmaxf(m_run[nt][1], mx1);
+      const float a0 = fast_exp2(m_run[nt][0] - mn0);
+      const float a1 = fast_exp2(m_run[nt][1] - mn1);
+      m_run[nt][0] = mn0;
+      m_run[nt][1] = mn1;
+      const float p0 = fast_exp2(s[0] - mn0);
+      const float p1 = fast_exp2(s[1] - mn1);
+      const float p2 = fast_exp2(s[2] - mn0);
+      const float p3 = fast_exp2(s[3] - mn1);
+      l_run[nt][0] = l_run[nt][0] * a0 + p0 + p2;
+      l_run[nt][1] = l_run[nt][1] * a1 + p1 + p3;
+#pragma unroll
+      for (int mt = 0; mt < F::kMTiles; ++mt) {
+        o[nt][mt][0] *= a0;
+        o[nt][mt][1] *= a1;
+        o[nt][mt][2] *= a0;
+        o[nt][mt][3] *= a1;
+      }
+      pb[nt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
+      pb[nt][1] = movmatrix_trans(pack_bf16x2(p2, p3));
+    }
+
+    // ---- O^T += V^T P^T ----
+#pragma unroll
+    for (int mt = 0; mt < F::kMTiles; ++mt) {
+      const int c = (D == 16) ? 0 : mt / 4;
+      const int qq = (D == 16) ? 0 : mt % 4;
+      const uint32_t w0 = vw[0][4 * c + qq], w1 = vw[1][4 * c + qq];
+      const uint32_t w2 = vw[2][4 * c + qq], w3 = vw[3][4 * c + qq];
+      const uint32_t a0 = prmt(w0, w1, 0x5410);
+      const uint32_t a1 = prmt(w0, w1, 0x7632);
+      const uint32_t a2 = prmt(w2, w3, 0x5410);
+      const uint32_t a3 = prmt(w2, w3, 0x7632);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_16816(o[nt][mt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+    }
+  }
+
+  // ---- merge the 4 warps of the CTA ----
+  // smem: m[4][G8], l[4][G8], O[4][G8][D] with G8 = 8*NT
+  constexpr int G8 = 8 * NT;
+  float* sm_m = smem;
+  float* sm_l = sm_m + kDecodeWarps * G8;
+  float* sm_o = sm_l + kDecodeWarps * G8;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float l0 = l_run[nt][0], l1 = l_run[nt][1];
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+    }
+    const int h0 = nt * 8 + 2 * t;
+    if (g == 0) {
+      sm_m[warp * G8 + h0] = m_run[nt][0];
+      sm_m[warp * G8 + h0 + 1] = m_run[nt][1];
+      sm_l[warp * G8 + h0] = l0;
+      sm_l[warp * G8 + h0 + 1] = l1;
+    }
+#pragma unroll
+    for (int mt = 0; mt < F::kMTiles; ++mt) {
+      // logical rows (mt, g) and (mt, g+8) -> physical d
+      int d0;
+      if constexpr (D == 16) {
+        d0 = 2 * g;
+      } else {
+        d0 = (mt / 4) * 64 + g * 8 + (mt % 4) * 2;
+      }
+      float* oh0 = sm_o + ((size_t)warp * G8 + h0) * D;
+      float* oh1 = oh0 + D;
+      oh0[d0] = o[nt][mt][0];
+      oh1[d0] = o[nt][mt][1];
+      oh0[d0 + 1] = o[nt][mt][2];
+      oh1[d0 + 1] = o[nt][mt][3];
+    }
+  }
+  __syncthreads();
+
+  const int hq0 = kvh * G;
+  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+    const int h = idx / D;
+    const int dd = idx - h * D;
+    float M = -CUDART_INF_F;
+#pragma unroll
+    for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, sm_m[w * G8 + h]);
+    float L = 0.f, O = 0.f;
+    if (M != -CUDART_INF_F) {
+#pragma unroll
+      for (int w = 0; w < kDecodeWarps; ++w) {
+        const float sc = fast_exp2(sm_m[w * G8 + h] - M);
+        L += sc * sm_l[w * G8 + h];
+        O += sc * sm_o[((size_t)w * G8 + h) * D + dd];
+      }
+    }
+    const size_t bh = (size_t)b * p.n_q_heads + hq0 + h;
+    if (p.n_splits == 1) {
+      store_out<OutT>(reinterpret_cast<OutT*>(p.out) + bh * D + dd, O / L);
+    } else {
+      p.ws_o[(bh * p.n_splits + split) * D + dd] = O;
+      if (dd == 0) {
+        p.ws_ml[(bh * p.n_splits + split) * 2 + 0] = M;
+        p.ws_ml[(bh * p.n_splits + split) * 2 + 1] = L;
+      }
+    }
+  }
+}
+
+// Merge of the per-split partials: grid (B * Hq), one thread per d.
+template <int D, typename OutT>
+__global__ void __launch_bounds__(D < 32 ? 32 : D)
+swa_decode_combine_kernel(const DecodeParams p) {
+  const size_t bh = blockIdx.x;
+  const int dd = threadIdx.x;
+  if (dd >= D) return;
+  const int S = p.n_splits;
+  const float* ml = p.ws_ml + bh * S * 2;
+  float M = -CUDART_INF_F;
+  for (int s = 0; s < S; ++s) M = fmaxf(M, ml[2 * s]);
+  float L = 0.f, O = 0.f;
+  const float* op = p.ws_o + bh * S * D + dd;
+  for (int s = 0; s < S; ++s) {
+    const float m = ml[2 * s];
+    if (m == -CUDART_INF_F) continue;
+    const float sc = fast_exp2(m - M);
+    L += sc * ml[2 * s + 1];
+    O += sc * op[(size_t)s * D];
+  }
+  store_out<OutT>(reinterpret_cast<OutT*>(p.out) + bh * D + dd, O / L);
+}
+
+namespace {
+
+template <int D, int NT, typename OutT>
+cudaError_t launch_decode_t(const DecodeParams& p, cudaStream_t stream) {
+  constexpr int G8 = 8 * NT;
+  const size_t smem = sizeof(float) * (size_t)kDecodeWarps * G8 * (2 + D);
+  auto kern = swa_decode_kernel<D, NT, OutT>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid(p.n_splits, p.n_kv_heads, p.batch);
+  kern<<<grid, kDecodeWarps * 32, smem, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || p.n_splits == 1) return e;
+  swa_decode_combine_kernel<D, OutT><<<(unsigned)((size_t)p.batch * p.n_q_heads), D < 32 ? 32 : D, 0,
+                                       stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <int D, typename OutT>
+cudaError_t launch_decode_d(const DecodeParams& p, cudaStream_t stream) {
+  const int G = p.n_q_heads / p.n_kv_heads;
+  if (G <= 8) return launch_decode_t<D, 1, OutT>(p, stream);
+  return launch_decode_t<D, 2, OutT>(p, stream);
+}
+
+template <typename OutT>
+cudaError_t launch_decode_o(const DecodeParams& p, cudaStream_t stream) {
+  switch (p.head_dim) {
+    case 16: return launch_decode_d<16, OutT>(p, stream);
+    case 64: return launch_decode_d<64, OutT>(p, stream);
+    case 128: return launch_decode_d<128, OutT>(p, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream) {
+  if (p.out_f32) return launch_decode_o<float>(p, stream);
+  return launch_decode_o<__nv_bfloat16>(p, stream);
+}
+
+}  // namespace swa

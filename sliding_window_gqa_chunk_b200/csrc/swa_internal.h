@@ -1,0 +1,77 @@
+// swa_internal.h - launch parameter blocks shared between the C-ABI layer
+// (swa_api.cu) and the kernel files.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace swa {
+
+struct AppendParams {
+  __nv_bfloat16* k_cache;       // [B][Hkv][W][d]
+  __nv_bfloat16* v_cache;
+  const __nv_bfloat16* k;       // [B][max_tokens][Hkv][d]
+  const __nv_bfloat16* v;
+  const int32_t* start_pos;     // device [B]
+  const int32_t* n_tokens;      // device [B]
+  int* status;                  // device status word
+  int batch, n_kv_heads, head_dim, window, max_tokens;
+};
+
+struct DecodeParams {
+  void* out;                    // [B][Hq][d] bf16 or f32
+  const __nv_bfloat16* q;       // [B][Hq][d]
+  const __nv_bfloat16* k_new;   // [B][Hkv][d]
+  const __nv_bfloat16* v_new;
+  const __nv_bfloat16* k_cache; // [B][Hkv][W][d] (read path)
+  const __nv_bfloat16* v_cache;
+  __nv_bfloat16* k_cache_w;     // same buffers (write of slot pos mod W)
+  __nv_bfloat16* v_cache_w;
+  const int32_t* pos;           // device [B]
+  float* ws_o;                  // [B][Hq][n_splits][d] partial O (n_splits > 1)
+  float* ws_ml;                 // [B][Hq][n_splits][2] partial (max, sum), log2 domain
+  int* status;
+  int batch, n_q_heads, n_kv_heads, head_dim, window;
+  int n_splits, slots_per_split;
+  float scale_log2;             // scale * log2(e)
+  int out_f32;
+};
+
+// Split of the W slots of one (sequence, kv head) across CTAs; depends only
+// on the shape so that the workspace size is a function of the dims.
+struct DecodeSplit {
+  int n_splits;
+  int slots_per_split;
+};
+DecodeSplit decode_split(int batch, int n_kv_heads, int window);
+
+struct PrefillParams {
+  void* out;                    // [B][max_tokens][Hq][d] bf16 or f32
+  const int32_t* start_pos;     // device [B]
+  const int32_t* n_tokens;      // device [B]
+  int* status;
+  int batch, n_q_heads, n_kv_heads, head_dim, window, max_tokens;
+  int heads_per_cta;            // 1 or 2 query heads of one kv group per CTA
+  int n_q_tiles;                // ceil(max_tokens / 128)
+  float scale_log2;
+  int out_f32;
+};
+
+// TMA descriptors of the prefill, built on the host per call.
+struct PrefillMaps {
+  CUtensorMap q;        // q [B][T][Hq][d]       box {d_box, 1, 128, 1}
+  CUtensorMap k;        // k [B][T][Hkv][d]
+  CUtensorMap v;
+  CUtensorMap kc;       // k_cache [B*Hkv][W][d] box {d_box, 128, 1}
+  CUtensorMap vc;
+};
+
+cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
+cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& maps, cudaStream_t stream);
+// TMA box width (elements of d per box row) and swizzle span used by the prefill kernel.
+void prefill_map_geometry(int head_dim, int* box_elems, int* swizzle_bytes);
+
+}  // namespace swa

@@ -1,0 +1,489 @@
+// swa_prefill.cu - attention of one prefill chunk over the rolling cache and the
+// chunk itself (Mistral 7B, section 2, Pre-fill and Chunking paragraph and
+// Figure 3), on the 5th-generation tensor cores of sm_100a.
+//
+// One CTA = one 128-row query tile of one or two query heads that share a kv
+// head (GQA: both heads reuse every K/V tile the CTA loads).  Warp roles:
+//   warps 0-3  softmax for head slot 0 (TMEM lanes 0-127 = the 128 query rows)
+//   warps 4-7  softmax for head slot 1
+//   warp  8    TMA producer (Q once, then K/V tiles into an NS-stage ring)
+//   warp  9    TMEM allocator and the single thread issuing tcgen05.mma
+// Per key tile j and head slot i:
+//   S_i = Q_i K_j^T       tcgen05.mma, A = Q (smem), B = K (smem), D = S_i (TMEM, fp32)
+//   softmax warps read S_i row by row (one thread per query row), mask, update
+//   the running max / sum (rescaling O_i only when the max grows by more than
+//   2^8), and write P_i = exp2(...) as bf16 back over S_i in TMEM
+//   O_i += P_i V_j        tcgen05.mma, A = P (TMEM), B = V (smem, d-contiguous)
+// Tensor memory: S_0 | S_1 | O_0 | O_1  (128 + 128 + d + d columns of 512).
+//
+// Key tiles: the keys of a chunk are the cache slots holding positions
+// [max(0, s + t_lo - W + 1), s) and the chunk rows [0, t_hi].  The cache
+// positions form one cyclic range of slots, so they are covered by 128-slot
+// tiles starting at slot-tile index first and wrapping past the last one: the
+// modular index p mod W goes straight into the TMA row coordinate.  Tiles that
+// no query row of the CTA can see are never loaded; inside the loaded tiles
+// each row masks the keys outside its own window [i - W + 1, i] and, in the
+// chunk, the keys after it (causal).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "swa_common.cuh"
+#include "swa_internal.h"
+#include "swa_tc.cuh"
+
+namespace swa {
+
+namespace {
+
+constexpr int kRows = 128;          // query rows per tile = TMEM lanes
+constexpr int kKeys = 128;          // keys per tile
+constexpr int kThreads = 320;       // 10 warps
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
+struct Cfg {
+  static constexpr int kSwzBytes = (D * 2 >= 128) ? 128 : D * 2;  // swizzle span = bytes per box row
+  static constexpr int kBoxD = kSwzBytes / 2;                      // d-elements per TMA box row
+  static constexpr int kColBlocks = (D * 2) / kSwzBytes;          // boxes per 128-row tile
+  static constexpr int kBlockBytes = kRows * kSwzBytes;           // one box
+  static constexpr int kTileBytes = kRows * D * 2;                // one 128 x d bf16 tile
+  static constexpr int kStages = (D == 128) ? 2 : 4;
+  static constexpr uint32_t kLayout = (kSwzBytes == 128) ? tc::kLayoutSW128 : tc::kLayoutSW32;
+  static constexpr int kSBO = 8 * kSwzBytes;                       // stride of 8-row groups
+  static constexpr int kKStepsPerBlock = kSwzBytes / 32;           // 16-element k-steps per box row
+  static constexpr int kSmemTiles = (2 + 2 * kStages) * kTileBytes;
+  static constexpr int kSmemBytes = kSmemTiles + 512 + 1024;       // barriers + alignment slack
+  static_assert(kColBlocks * kSwzBytes == D * 2, "head_dim must fill whole swizzle rows");
+};
+
+// The key tiles of one CTA, in issue order: cache tiles (cyclic over slot
+// tiles), then chunk tiles 0..qt.  Every role evaluates the same plan.
+struct TilePlan {
+  int n_cache;
+  int first_cache;
+  int n_wtiles;
+  int n_chunk;
+  __device__ __forceinline__ int total() const { return n_cache + n_chunk; }
+  __device__ __forceinline__ void at(int j, bool& is_cache, int& base) const {
+    if (j < n_cache) {
+      int ti = first_cache + j;
+      if (ti >= n_wtiles) ti -= n_wtiles;
+      is_cache = true;
+      base = ti * kKeys;
+    } else {
+      is_cache = false;
+      base = (j - n_cache) * kKeys;
+    }
+  }
+};
+
+__device__ __forceinline__ TilePlan make_plan(long long s, int t_lo, int qt, int W) {
+  TilePlan pl;
+  pl.n_wtiles = (W + kKeys - 1) / kKeys;
+  pl.n_chunk = qt + 1;
+  long long c_lo = s + t_lo - W + 1;
+  if (c_lo < 0) c_lo = 0;
+  const long long n_c = s - c_lo;  // cache positions some row of the tile can see
+  if (n_c <= 0) {
+    pl.n_cache = 0;
+    pl.first_cache = 0;
+    return pl;
+  }
+  const int a = (int)(c_lo % W);
+  const int last = (int)((c_lo + n_c - 1) % W);
+  const int ft = a / kKeys, lt = last / kKeys;
+  if (a + n_c <= W) {
+    pl.first_cache = ft;
+    pl.n_cache = lt - ft + 1;
+  } else if (lt < ft) {
+    pl.first_cache = ft;
+    pl.n_cache = (pl.n_wtiles - ft) + lt + 1;
+  } else {
+    pl.first_cache = 0;
+    pl.n_cache = pl.n_wtiles;
+  }
+  return pl;
+}
+
+template <typename OutT>
+__device__ __forceinline__ void store16(OutT* dst, const float (&v)[16], float scale);
+
+template <>
+__device__ __forceinline__ void store16<float>(float* dst, const float (&v)[16], float scale) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    d4[i] = make_float4(v[4 * i] * scale, v[4 * i + 1] * scale, v[4 * i + 2] * scale,
+                        v[4 * i + 3] * scale);
+}
+
+template <>
+__device__ __forceinline__ void store16<__nv_bfloat16>(__nv_bfloat16* dst, const float (&v)[16],
+                                                       float scale) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * i + 0] * scale, v[8 * i + 1] * scale);
+    w.y = pack_bf16x2(v[8 * i + 2] * scale, v[8 * i + 3] * scale);
+    w.z = pack_bf16x2(v[8 * i + 4] * scale, v[8 * i + 5] * scale);
+    w.w = pack_bf16x2(v[8 * i + 6] * scale, v[8 * i + 7] * scale);
+    d4[i] = w;
+  }
+}
+
+}  // namespace
+
+template <int D, typename OutT>
+__global__ void __launch_bounds__(kThreads, 1)
+swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps maps) {
+  using C = Cfg<D>;
+  constexpr int NS = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int qt = blockIdx.x;
+  const int b = blockIdx.z;
+  const int hpc = p.heads_per_cta;
+  const int G = p.n_q_heads / p.n_kv_heads;
+  const int pairs = G / hpc;
+  const int kvh = blockIdx.y / pairs;
+  const int h_first = kvh * G + (blockIdx.y % pairs) * hpc;
+  const int W = p.window;
+
+  const long long s = p.start_pos[b];
+  const int n = p.n_tokens[b];
+  if (s < 0 || n < 0 || n > p.max_tokens) {
+    if (threadIdx.x == 0 && qt == 0 && blockIdx.y == 0) raise_status(p.status, SWA_ERR_DEVICE_ARG);
+    return;
+  }
+  const int t_lo = qt * kRows;
+  if (t_lo >= n) return;  // whole CTA: nothing of this sequence in the tile
+  const TilePlan plan = make_plan(s, t_lo, qt, W);
+  const int n_tiles = plan.total();
+
+  // ---- shared memory carve-up (1024-byte aligned for the 128B swizzle) ----
+  const uint32_t raw_addr = tc::smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw_addr);
+  const uint32_t sQ = base;                                   // 2 tiles
+  const uint32_t sK = base + 2 * C::kTileBytes;               // NS tiles
+  const uint32_t sV = sK + NS * C::kTileBytes;                // NS tiles
+  const uint32_t sBar = base + C::kSmemTiles;
+  // barrier addresses (8 bytes each)
+  const uint32_t bar_q_full = sBar;
+  const uint32_t bar_k_full = sBar + 8;                // [NS]
+  const uint32_t bar_v_full = bar_k_full + 8 * NS;     // [NS]
+  const uint32_t bar_kv_empty = bar_v_full + 8 * NS;   // [NS]
+  const uint32_t bar_s_full = bar_kv_empty + 8 * NS;   // [2]
+  const uint32_t bar_p_full = bar_s_full + 16;         // [2]
+  const uint32_t bar_o_full = bar_p_full + 16;         // [2]
+  const uint32_t bar_done = bar_o_full + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::kSmemTiles + 256);
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(bar_q_full, 1);
+    for (int i = 0; i < NS; ++i) {
+      tc::mbar_init(bar_k_full + 8 * i, 1);
+      tc::mbar_init(bar_v_full + 8 * i, 1);
+      tc::mbar_init(bar_kv_empty + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(bar_s_full + 8 * i, 1);
+      tc::mbar_init(bar_p_full + 8 * i, kRows);
+      tc::mbar_init(bar_o_full + 8 * i, 1);
+    }
+    tc::mbar_init(bar_done, 1);
+    tc::mbar_fence_init();
+  }
+  if (warp == kMmaWarp) {
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kProducerWarp) {
+    // ============================ TMA producer ============================
+    if (lane == 0) {
+      tc::prefetch_map(&maps.q);
+      tc::prefetch_map(&maps.k);
+      tc::prefetch_map(&maps.v);
+      tc::prefetch_map(&maps.kc);
+      tc::prefetch_map(&maps.vc);
+      tc::mbar_arrive_expect_tx(bar_q_full, hpc * C::kTileBytes);
+      for (int i = 0; i < hpc; ++i)
+        for (int cb = 0; cb < C::kColBlocks; ++cb)
+          tc::tma_load_4d(sQ + i * C::kTileBytes + cb * C::kBlockBytes, &maps.q, cb * C::kBoxD,
+                          h_first + i, t_lo, b, bar_q_full);
+      bool ok = true;
+      for (int j = 0; j < n_tiles && ok; ++j) {
+        const int st = j % NS;
+        if (j >= NS) ok = tc::mbar_wait(bar_kv_empty + 8 * st, ((j / NS) - 1) & 1, p.status);
+        if (!ok) break;
+        bool is_cache;
+        int kbase;
+        plan.at(j, is_cache, kbase);
+        const uint32_t kdst = sK + st * C::kTileBytes;
+        const uint32_t vdst = sV + st * C::kTileBytes;
+        tc::mbar_arrive_expect_tx(bar_k_full + 8 * st, C::kTileBytes);
+        for (int cb = 0; cb < C::kColBlocks; ++cb) {
+          if (is_cache)
+            tc::tma_load_3d(kdst + cb * C::kBlockBytes, &maps.kc, cb * C::kBoxD, kbase,
+                            b * p.n_kv_heads + kvh, bar_k_full + 8 * st);
+          else
+            tc::tma_load_4d(kdst + cb * C::kBlockBytes, &maps.k, cb * C::kBoxD, kvh, kbase, b,
+                            bar_k_full + 8 * st);
+        }
+        tc::mbar_arrive_expect_tx(bar_v_full + 8 * st, C::kTileBytes);
+        for (int cb = 0; cb < C::kColBlocks; ++cb) {
+          if (is_cache)
+            tc::tma_load_3d(vdst + cb * C::kBlockBytes, &maps.vc, cb * C::kBoxD, kbase,
+                            b * p.n_kv_heads + kvh, bar_v_full + 8 * st);
+          else
+            tc::tma_load_4d(vdst + cb * C::kBlockBytes, &maps.v, cb * C::kBoxD, kvh, kbase, b,
+                            bar_v_full + 8 * st);
+        }
+      }
+      // Before leaving, make sure no copy issued here is still in flight.
+      tc::mbar_wait(bar_q_full, 0, p.status);
+      const int j0 = n_tiles > NS ? n_tiles - NS : 0;
+      for (int j = j0; j < n_tiles; ++j) {
+        tc::mbar_wait(bar_k_full + 8 * (j % NS), (j / NS) & 1, p.status);
+        tc::mbar_wait(bar_v_full + 8 * (j % NS), (j / NS) & 1, p.status);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ============================ MMA issuer ============================
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = tc::make_idesc_bf16(kRows, kKeys, false, false);
+      constexpr uint32_t idesc_pv = tc::make_idesc_bf16(kRows, D, false, true);
+      auto issue_s = [&](int i, int st) {
+        const uint32_t d_tmem = tmem + i * kKeys;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const int cb = ks / C::kKStepsPerBlock;
+          const int kin = ks % C::kKStepsPerBlock;
+          const uint32_t off = cb * C::kBlockBytes + kin * 32;
+          const uint64_t ad = tc::make_sdesc(sQ + i * C::kTileBytes + off, 16, C::kSBO, C::kLayout);
+          const uint64_t bd = tc::make_sdesc(sK + st * C::kTileBytes + off, 16, C::kSBO, C::kLayout);
+          tc::mma_ss(d_tmem, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int i, int st, bool accumulate) {
+        const uint32_t d_tmem = tmem + 2 * kKeys + i * D;
+        const uint32_t a_tmem = tmem + i * kKeys;
+#pragma unroll
+        for (int ks = 0; ks < kKeys / 16; ++ks) {
+          const uint64_t bd = tc::make_sdesc(sV + st * C::kTileBytes + ks * 16 * C::kSwzBytes,
+                                             C::kBlockBytes, C::kSBO, C::kLayout);
+          tc::mma_ts(d_tmem, a_tmem + ks * 8, bd, idesc_pv, (accumulate || ks > 0) ? 1u : 0u);
+        }
+      };
+
+      bool ok = tc::mbar_wait(bar_q_full, 0, p.status);
+      tc::tc_fence_after();
+      for (int j = 0; j < n_tiles && ok; ++j) {
+        const int st = j % NS;
+        ok = tc::mbar_wait(bar_k_full + 8 * st, (j / NS) & 1, p.status);
+        if (!ok) break;
+        tc::tc_fence_after();
+        for (int i = 0; i < hpc && ok; ++i) {
+          if (j > 0) {
+            const int sp = (j - 1) % NS;
+            ok = tc::mbar_wait(bar_p_full + 8 * i, (j - 1) & 1, p.status);
+            if (ok && i == 0) ok = tc::mbar_wait(bar_v_full + 8 * sp, ((j - 1) / NS) & 1, p.status);
+            if (!ok) break;
+            tc::tc_fence_after();
+            issue_pv(i, sp, j - 1 > 0);
+          }
+          issue_s(i, st);
+          tc::tc_commit(bar_s_full + 8 * i);
+        }
+        if (ok && j > 0) tc::tc_commit(bar_kv_empty + 8 * ((j - 1) % NS));
+      }
+      if (ok) {
+        const int jl = n_tiles - 1;
+        const int sl = jl % NS;
+        for (int i = 0; i < hpc && ok; ++i) {
+          ok = tc::mbar_wait(bar_p_full + 8 * i, jl & 1, p.status);
+          if (ok && i == 0) ok = tc::mbar_wait(bar_v_full + 8 * sl, (jl / NS) & 1, p.status);
+          if (!ok) break;
+          tc::tc_fence_after();
+          issue_pv(i, sl, jl > 0);
+          tc::tc_commit(bar_o_full + 8 * i);
+        }
+      }
+      // All MMAs must have finished before the TMEM is released.
+      tc::tc_commit(bar_done);
+      tc::mbar_wait(bar_done, 0, p.status);
+    }
+  } else if (warp / 4 < hpc) {
+    // ============================ softmax / epilogue ============================
+    const int i = warp / 4;                   // head slot
+    const int row = (warp % 4) * 32 + lane;   // query row within the tile = TMEM lane
+    const int t = t_lo + row;                 // chunk row
+    const long long pos_i = s + t;            // absolute query position
+    const uint32_t lane_addr = (uint32_t)((warp % 4) * 32) << 16;
+    const uint32_t tS = tmem + lane_addr + i * kKeys;
+    const uint32_t tO = tmem + lane_addr + 2 * kKeys + i * D;
+    const float sl2 = p.scale_log2;
+    // this row's visible cache slots: the cyclic range [a_i, a_i + len_i)
+    long long lo_i = pos_i - W + 1;
+    if (lo_i < 0) lo_i = 0;
+    const int len_i = (int)(s - lo_i);          // <= W - 1; <= 0 means none
+    const int a_i = (int)(lo_i % W);
+
+    float m_run = -CUDART_INF_F;
+    float l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      ok = tc::mbar_wait(bar_s_full + 8 * i, j & 1, p.status);
+      if (!ok) break;
+      tc::tc_fence_after();
+      float sv[kKeys];
+      {
+        float* chunk = sv;
+#pragma unroll
+        for (int c = 0; c < kKeys / 32; ++c)
+          tc::tmem_ld32(tS + c * 32, *reinterpret_cast<float(*)[32]>(chunk + c * 32));
+      }
+      tc::tc_wait_ld();
+#pragma unroll
+      for (int c = 0; c < kKeys / 16; ++c) tc::reg_fence16(sv + c * 16);
+
+      bool is_cache;
+      int kbase;
+      plan.at(j, is_cache, kbase);
+      if (is_cache) {
+        int d0 = kbase - a_i;
+        if (d0 < 0) d0 += W;
+        const bool full = (kbase + kKeys <= W) && (len_i > 0) && (d0 + kKeys <= len_i);
+        if (!full) {
+#pragma unroll
+          for (int k = 0; k < kKeys; ++k) {
+            const int r = kbase + k;
+            int dd = r - a_i;
+            if (dd < 0) dd += W;
+            const bool vis = (r < W) && (dd < len_i);
+            if (!vis) sv[k] = -CUDART_INF_F;
+          }
+        }
+      } else {
+        if (kbase + kKeys - 1 > t) {
+#pragma unroll
+          for (int k = 0; k < kKeys; ++k)
+            if (kbase + k > t) sv[k] = -CUDART_INF_F;
+        }
+      }
+
+      float mx = sv[0];
+#pragma unroll
+      for (int k = 1; k < kKeys; ++k) mx = fmaxf(mx, sv[k]);
+      const float m_new = fmaxf(m_run, mx * sl2);
+      if (m_new > m_run + kRescaleThreshold) {
+        const float alpha = fast_exp2(m_run - m_new);  // 0 while nothing was visible yet
+        if (j > 0) {
+          // O_i holds the previous tiles' sum (its last PV finished before S_i(j) did)
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) {
+            float ov[16];
+            tc::tmem_ld16(tO + c * 16, ov);
+            tc::tc_wait_ld();
+            tc::reg_fence16(ov);
+            uint32_t ow[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) ow[e] = __float_as_uint(ov[e] * alpha);
+            tc::tmem_st16(tO + c * 16, ow);
+          }
+        }
+        l_run *= alpha;
+        m_run = m_new;
+      }
+      const float nb = (m_run == -CUDART_INF_F) ? 0.f : -m_run;
+#pragma unroll
+      for (int c = 0; c < kKeys / 32; ++c) {
+        uint32_t pw[16];
+#pragma unroll
+        for (int w = 0; w < 16; ++w) {
+          const float p0 = fast_exp2(fmaf(sv[c * 32 + 2 * w], sl2, nb));
+          const float p1 = fast_exp2(fmaf(sv[c * 32 + 2 * w + 1], sl2, nb));
+          l_run += p0 + p1;
+          pw[w] = pack_bf16x2(p0, p1);
+        }
+        tc::tmem_st16(tS + c * 16, pw);  // P (bf16 pairs) over the first 64 columns of S_i
+      }
+      tc::tc_wait_st();
+      tc::tc_fence_before();
+      tc::mbar_arrive(bar_p_full + 8 * i);
+    }
+
+    if (ok) ok = tc::mbar_wait(bar_o_full + 8 * i, 0, p.status);
+    if (ok) {
+      tc::tc_fence_after();
+      const float inv_l = 1.f / l_run;
+      OutT* dst = reinterpret_cast<OutT*>(p.out) +
+                  (((size_t)b * p.max_tokens + t) * p.n_q_heads + (h_first + i)) * D;
+#pragma unroll
+      for (int c = 0; c < D / 16; ++c) {
+        float ov[16];
+        tc::tmem_ld16(tO + c * 16, ov);
+        tc::tc_wait_ld();
+        tc::reg_fence16(ov);
+        if (t < n) store16<OutT>(dst + c * 16, ov, inv_l);
+      }
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+namespace {
+
+template <int D, typename OutT>
+cudaError_t launch_prefill_t(const PrefillParams& p, const PrefillMaps& maps, cudaStream_t stream) {
+  using C = Cfg<D>;
+  auto kern = swa_prefill_kernel<D, OutT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.n_q_tiles, p.n_q_heads / p.heads_per_cta, p.batch);
+  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(p, maps);
+  return cudaGetLastError();
+}
+
+template <typename OutT>
+cudaError_t launch_prefill_o(const PrefillParams& p, const PrefillMaps& maps, cudaStream_t stream) {
+  switch (p.head_dim) {
+    case 16: return launch_prefill_t<16, OutT>(p, maps, stream);
+    case 64: return launch_prefill_t<64, OutT>(p, maps, stream);
+    case 128: return launch_prefill_t<128, OutT>(p, maps, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+void prefill_map_geometry(int head_dim, int* box_elems, int* swizzle_bytes) {
+  const int swz = (head_dim * 2 >= 128) ? 128 : head_dim * 2;
+  *swizzle_bytes = swz;
+  *box_elems = swz / 2;
+}
+
+cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& maps, cudaStream_t stream) {
+  if (p.out_f32) return launch_prefill_o<float>(p, maps, stream);
+  return launch_prefill_o<__nv_bfloat16>(p, maps, stream);
+}
+
+}  // namespace swa

@@ -1,0 +1,73 @@
+"""Shared pieces of the GPU parity tests: running the CUDA path through the
+Python binding of the C ABI, and the tolerance check against the oracle.
+
+Tolerances (the same as the pass bar for attention outputs from bf16 inputs
+with fp32 accumulation): max |gpu - ref| <= 1e-2 and
+sum |gpu - ref| / sum |ref| <= 2e-3, with fp32 outputs.  bf16 outputs carry
+one more rounding (relative 2^-9) and are held to 1e-2 / 4e-3.
+"""
+import numpy as np
+import torch
+
+import sliding_window_gqa_chunk_b200 as swa
+
+MAX_ABS = 1e-2
+REL_L1 = 2e-3
+REL_L1_BF16_OUT = 4e-3
+
+
+def rel_l1(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    return float(np.abs(got - ref).sum() / max(np.abs(ref).sum(), 1e-300))
+
+
+def assert_close(got, ref, what="", bf16_out=False):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    err = np.abs(got - ref)
+    mx = float(err.max()) if err.size else 0.0
+    rl = rel_l1(got, ref)
+    bar = REL_L1_BF16_OUT if bf16_out else REL_L1
+    assert mx <= MAX_ABS and rl <= bar, f"{what}: max_abs={mx:.3e} rel_l1={rl:.3e}"
+    return mx, rl
+
+
+def dev_i32(values, device="cuda"):
+    return torch.tensor([int(x) for x in values], dtype=torch.int32, device=device)
+
+
+def gpu_chunked_prefill(dims, q, k, v, lengths, chunk, device="cuda"):
+    """Prefill padded prompts q/k/v [B, L, H, d] (bf16, CPU) chunk by chunk on
+    the GPU.  Returns (out [B, L, Hq, d] float64 numpy, k_cache, v_cache)."""
+    B, L, Hq, d = q.shape
+    kc, vc = swa.new_cache(dims, device)
+    out = torch.zeros((B, L, Hq, d), dtype=torch.float64)
+    n_calls = max((n + chunk - 1) // chunk for n in lengths)
+    for c in range(n_calls):
+        st = c * chunk
+        counts = [max(0, min(chunk, n - st)) for n in lengths]
+        hi = min(L, st + chunk)
+        T = chunk
+        qc = torch.zeros((B, T, Hq, d), dtype=torch.bfloat16)
+        kc_in = torch.zeros((B, T, k.shape[2], d), dtype=torch.bfloat16)
+        vc_in = torch.zeros((B, T, k.shape[2], d), dtype=torch.bfloat16)
+        qc[:, : hi - st] = q[:, st:hi]
+        kc_in[:, : hi - st] = k[:, st:hi]
+        vc_in[:, : hi - st] = v[:, st:hi]
+        qg, kg, vg = qc.to(device), kc_in.to(device), vc_in.to(device)
+        o = torch.zeros((B, T, Hq, d), dtype=dims.torch_out_dtype, device=device)
+        sp = dev_i32([st] * B, device)
+        nt = dev_i32(counts, device)
+        swa.prefill_chunk(dims, o, qg, kg, vg, kc, vc, sp, nt)
+        swa.cache_append(dims, kc, vc, kg, vg, sp, nt)
+        out[:, st:hi] = o[:, : hi - st].double().cpu()
+    torch.cuda.synchronize()
+    swa.device_status()
+    return out.numpy(), kc, vc
+
+
+def cache_as_f64(kc):
+    return kc.double().cpu().numpy()

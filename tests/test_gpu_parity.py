@@ -1,0 +1,261 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Bit-exact: cache slot placement (the cache bytes after every append / decode)
+and the mask (zero-Q / one-hot-V probe).  Within tolerance (tests/gpu_helpers):
+attention outputs.  Shapes span several 128-row tiles, ragged tails, windows
+that are not multiples of 128 or smaller than one tile, chunks shorter than
+the window (so cache tiles wrap), GQA group sizes 1, 2, 3, 4 and 8, and head
+dims 16, 64 and 128.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sliding_window_gqa_chunk_b200 as swa
+from swa_workloads import random_case, tiny_inputs, TINY_PREFILL, TINY_SHAPE
+from tests.gpu_helpers import (assert_close, cache_as_f64, dev_i32, gpu_chunked_prefill)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def mk_dims(B, Hq, Hkv, d, W, scale=None, out="f32"):
+    return swa.Dims(B, Hq, Hkv, d, W, scale if scale is not None else 1.0 / math.sqrt(d), out)
+
+
+# ----------------------------------------------------------------------------
+# Cache append: slot placement is bit-exact
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d", [16, 64, 128])
+def test_append_slot_placement_bit_exact(d):
+    B, Hkv, W, T = 3, 2, 64, 40
+    dims = mk_dims(B, 4, Hkv, d, W)
+    kc, vc = swa.new_cache(dims, DEV)
+    ref = oracle.RollingCache(B, Hkv, W, d)
+    g = torch.Generator().manual_seed(d)
+    calls = [([0, 10, 50], [40, 7, 30]), ([40, 17, 80], [24, 40, 0]), ([64, 57, 80], [1, 33, 39])]
+    for starts, counts in calls:
+        k = torch.randn(B, T, Hkv, d, generator=g).to(torch.bfloat16)
+        v = torch.randn(B, T, Hkv, d, generator=g).to(torch.bfloat16)
+        swa.cache_append(dims, kc, vc, k.to(DEV), v.to(DEV), dev_i32(starts), dev_i32(counts))
+        oracle.cache_append(ref, k, v, starts, counts)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(cache_as_f64(kc), ref.k)
+        np.testing.assert_array_equal(cache_as_f64(vc), ref.v)
+    swa.device_status()
+
+
+# ----------------------------------------------------------------------------
+# Config 1: 3 chunks of 4 with W = 4, then 4 decode steps
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("out_dtype", ["f32", "bf16"])
+def test_tiny_workload_prefill_then_decode(out_dtype):
+    s = TINY_SHAPE
+    dims = swa.Dims(1, s.n_q_heads, s.n_kv_heads, s.head_dim, s.window, TINY_PREFILL.scale,
+                    out_dtype)
+    chunks, steps = tiny_inputs()
+    kc, vc = swa.new_cache(dims, DEV)
+    ref = oracle.RollingCache(1, s.n_kv_heads, s.window, s.head_dim)
+    bf = out_dtype == "bf16"
+    for c, (q, k, v) in enumerate(chunks):
+        st = 4 * c
+        o = torch.zeros((1, 4, s.n_q_heads, s.head_dim), dtype=dims.torch_out_dtype, device=DEV)
+        sp, nt = dev_i32([st]), dev_i32([4])
+        swa.prefill_chunk(dims, o, q.to(DEV), k.to(DEV), v.to(DEV), kc, vc, sp, nt)
+        swa.cache_append(dims, kc, vc, k.to(DEV), v.to(DEV), sp, nt)
+        expect = oracle.prefill_chunk(ref, q, k, v, [st], [4], dims.scale)
+        oracle.cache_append(ref, k, v, [st], [4])
+        assert_close(o.double().cpu().numpy(), expect, f"chunk {c}", bf16_out=bf)
+        np.testing.assert_array_equal(cache_as_f64(kc), ref.k)
+        np.testing.assert_array_equal(cache_as_f64(vc), ref.v)
+    ws = torch.empty(swa.decode_workspace_size(dims), dtype=torch.uint8, device=DEV)
+    for i, (q, k, v) in enumerate(steps):
+        p = 12 + i
+        o = torch.zeros((1, s.n_q_heads, s.head_dim), dtype=dims.torch_out_dtype, device=DEV)
+        swa.decode(dims, o, q.to(DEV), k.to(DEV), v.to(DEV), kc, vc, dev_i32([p]), ws)
+        expect = oracle.decode(ref, q, k, v, [p], dims.scale)
+        assert_close(o.double().cpu().numpy(), expect, f"step {i}", bf16_out=bf)
+        np.testing.assert_array_equal(cache_as_f64(kc), ref.k)
+        np.testing.assert_array_equal(cache_as_f64(vc), ref.v)
+    # positions 12..15 went to slots 0..3
+    np.testing.assert_array_equal(ref.pos[0], [12, 13, 14, 15])
+    swa.device_status()
+
+
+# ----------------------------------------------------------------------------
+# Mask structure: zero-Q / one-hot-V probe, bit-exact support
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("W,chunk,L,d,Hq,Hkv", [(4, 4, 12, 16, 4, 2), (8, 8, 24, 64, 4, 1),
+                                               (8, 5, 23, 64, 2, 2), (16, 16, 120, 128, 8, 2)])
+def test_mask_probe_support_bit_exact(W, chunk, L, d, Hq, Hkv):
+    """Q = 0 gives equal weights on the visible keys, V = one-hot(position mod d)
+    marks them: the set of non-zero output columns is the visible set."""
+    g = torch.Generator().manual_seed(W * 100 + L)
+    q = torch.zeros(1, L, Hq, d, dtype=torch.bfloat16)
+    k = torch.randn(1, L, Hkv, d, generator=g).to(torch.bfloat16)
+    v = torch.zeros(1, L, Hkv, d, dtype=torch.bfloat16)
+    for p in range(L):
+        v[0, p, :, p % d] = 1.0
+    dims = mk_dims(1, Hq, Hkv, d, W, scale=1.0)
+    got, _, _ = gpu_chunked_prefill(dims, q, k, v, [L], chunk)
+    ref, _ = oracle.run_chunked_prefill(q, k, v, W, chunk, 1.0)
+    np.testing.assert_array_equal(got != 0, ref != 0)
+    # and each row sees min(i + 1, W) keys when positions are distinct mod d
+    if L <= d:
+        counts = (got[0, :, 0] != 0).sum(-1)
+        np.testing.assert_array_equal(counts, np.minimum(np.arange(L) + 1, W))
+
+
+# ----------------------------------------------------------------------------
+# Prefill against the oracle on random inputs
+# ----------------------------------------------------------------------------
+
+PREFILL_CASES = [
+    # B, lengths,     W,   chunk, Hq, Hkv, d
+    (1, [300],        128, 128,   4,  2,   128),
+    (2, [700, 333],   256, 256,   8,  2,   64),
+    (1, [520],        512, 512,   2,  2,   128),   # G = 1
+    (2, [390, 129],   200, 200,   6,  2,   64),    # G = 3, W not a multiple of 128
+    (1, [64],         32,  32,    8,  1,   16),    # G = 8, W below one tile
+    (2, [600, 411],   256, 100,   4,  2,   128),   # chunk < W: wrapping cache tiles
+    (3, [257, 1, 130], 384, 384,  4,  1,   128),   # ragged, a 1-token prompt
+]
+
+
+@pytest.mark.parametrize("B,lengths,W,chunk,Hq,Hkv,d", PREFILL_CASES)
+def test_prefill_matches_oracle(B, lengths, W, chunk, Hq, Hkv, d):
+    L = max(lengths)
+    q, k, v = random_case(1000 + W + chunk + d, B, L, Hq, Hkv, d, lengths=lengths)
+    dims = mk_dims(B, Hq, Hkv, d, W)
+    got, kc, vc = gpu_chunked_prefill(dims, q, k, v, lengths, chunk)
+    ref, rcache = oracle.run_chunked_prefill(q, k, v, W, chunk, dims.scale, lengths=lengths)
+    assert_close(got, ref, f"prefill B={B} L={lengths} W={W} chunk={chunk}")
+    np.testing.assert_array_equal(cache_as_f64(kc), rcache.k)
+    np.testing.assert_array_equal(cache_as_f64(vc), rcache.v)
+
+
+def test_prefill_bf16_output():
+    B, L, W, Hq, Hkv, d = 2, 300, 128, 8, 2, 128
+    q, k, v = random_case(77, B, L, Hq, Hkv, d)
+    dims = mk_dims(B, Hq, Hkv, d, W, out="bf16")
+    got, _, _ = gpu_chunked_prefill(dims, q, k, v, [L, L], W)
+    ref, _ = oracle.run_chunked_prefill(q, k, v, W, W, dims.scale)
+    assert_close(got, ref, "bf16 out", bf16_out=True)
+
+
+def test_prefill_chunk_after_decode_steps():
+    """A chunk that starts at a position that is not a multiple of 128, after a
+    few decode steps, with a cache that is not full yet (unwritten slots are zero)."""
+    B, W, Hq, Hkv, d = 2, 256, 4, 2, 128
+    first, T = 37, 200
+    L = first + T
+    q, k, v = random_case(55, B, L, Hq, Hkv, d)
+    dims = mk_dims(B, Hq, Hkv, d, W)
+    kc, vc = swa.new_cache(dims, DEV)
+    ref = oracle.RollingCache(B, Hkv, W, d)
+    ws = torch.empty(swa.decode_workspace_size(dims), dtype=torch.uint8, device=DEV)
+    for p in range(first):
+        o = torch.zeros((B, Hq, d), dtype=torch.float32, device=DEV)
+        swa.decode(dims, o, q[:, p].contiguous().to(DEV), k[:, p].contiguous().to(DEV),
+                   v[:, p].contiguous().to(DEV), kc, vc, dev_i32([p] * B), ws)
+        expect = oracle.decode(ref, q[:, p], k[:, p], v[:, p], [p] * B, dims.scale)
+        assert_close(o.double().cpu().numpy(), expect, f"decode {p}")
+    o = torch.zeros((B, T, Hq, d), dtype=torch.float32, device=DEV)
+    qc, kcn, vcn = (x[:, first:].contiguous() for x in (q, k, v))
+    sp, nt = dev_i32([first] * B), dev_i32([T, T - 50])
+    swa.prefill_chunk(dims, o, qc.to(DEV), kcn.to(DEV), vcn.to(DEV), kc, vc, sp, nt)
+    swa.cache_append(dims, kc, vc, kcn.to(DEV), vcn.to(DEV), sp, nt)
+    expect = oracle.prefill_chunk(ref, qc, kcn, vcn, [first] * B, [T, T - 50], dims.scale)
+    oracle.cache_append(ref, kcn, vcn, [first] * B, [T, T - 50])
+    assert_close(o.double().cpu().numpy(), expect, "chunk after decode")
+    np.testing.assert_array_equal(cache_as_f64(kc), ref.k)
+    swa.device_status()
+
+
+# ----------------------------------------------------------------------------
+# Decode against the oracle
+# ----------------------------------------------------------------------------
+
+DECODE_CASES = [
+    # B, W,    Hq, Hkv, d,   first positions, steps
+    (4, 4096, 32, 8, 128, [4096, 5000, 9999, 31000], 3),
+    (2, 300, 8, 2, 64, [0, 298], 4),          # empty cache / fills exactly at W-1
+    (3, 100, 12, 4, 128, [5, 99, 100000], 3),  # G = 3, far position
+    (1, 16, 16, 1, 16, [3], 20),               # G = 16, wraps several times
+    (5, 1000, 4, 4, 64, [0, 1, 2, 999, 1000], 2),  # G = 1
+    (2, 4096, 64, 8, 128, [70000, 4095], 2),   # G = 8
+]
+
+
+@pytest.mark.parametrize("B,W,Hq,Hkv,d,pos0,steps", DECODE_CASES)
+def test_decode_matches_oracle(B, W, Hq, Hkv, d, pos0, steps):
+    g = torch.Generator().manual_seed(B * 1000 + W + d)
+    dims = mk_dims(B, Hq, Hkv, d, W)
+    # start from a cache holding positions [max(0, p - W), p) for each sequence
+    kc = torch.zeros(B, Hkv, W, d, dtype=torch.bfloat16)
+    vc = torch.zeros_like(kc)
+    ref = oracle.RollingCache(B, Hkv, W, d)
+    for b, p0 in enumerate(pos0):
+        for p in range(max(0, p0 - W), p0):
+            kr = torch.randn(Hkv, d, generator=g).to(torch.bfloat16)
+            vr = torch.randn(Hkv, d, generator=g).to(torch.bfloat16)
+            kc[b, :, p % W] = kr
+            vc[b, :, p % W] = vr
+            ref.write(b, p, kr, vr)
+    kc, vc = kc.to(DEV), vc.to(DEV)
+    ws = torch.empty(swa.decode_workspace_size(dims), dtype=torch.uint8, device=DEV)
+    for s in range(steps):
+        pos = [p + s for p in pos0]
+        q = torch.randn(B, Hq, d, generator=g).to(torch.bfloat16)
+        k = torch.randn(B, Hkv, d, generator=g).to(torch.bfloat16)
+        v = torch.randn(B, Hkv, d, generator=g).to(torch.bfloat16)
+        o = torch.zeros((B, Hq, d), dtype=torch.float32, device=DEV)
+        swa.decode(dims, o, q.to(DEV), k.to(DEV), v.to(DEV), kc, vc, dev_i32(pos), ws)
+        expect = oracle.decode(ref, q, k, v, pos, dims.scale)
+        assert_close(o.double().cpu().numpy(), expect, f"decode step {s}")
+        np.testing.assert_array_equal(cache_as_f64(kc), ref.k)
+        np.testing.assert_array_equal(cache_as_f64(vc), ref.v)
+    swa.device_status()
+
+
+def test_decode_bf16_output():
+    B, W, Hq, Hkv, d = 3, 512, 32, 8, 128
+    g = torch.Generator().manual_seed(9)
+    dims = mk_dims(B, Hq, Hkv, d, W, out="bf16")
+    kc = torch.randn(B, Hkv, W, d, generator=g).to(torch.bfloat16)
+    vc = torch.randn(B, Hkv, W, d, generator=g).to(torch.bfloat16)
+    ref = oracle.RollingCache(B, Hkv, W, d)
+    pos = [600, 1023, 5000]
+    for b in range(B):
+        for p in range(pos[b] - W, pos[b]):
+            ref.write(b, p, kc[b, :, p % W], vc[b, :, p % W])
+    q = torch.randn(B, Hq, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, Hkv, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, Hkv, d, generator=g).to(torch.bfloat16)
+    kcd, vcd = kc.to(DEV), vc.to(DEV)
+    ws = torch.empty(swa.decode_workspace_size(dims), dtype=torch.uint8, device=DEV)
+    o = torch.zeros((B, Hq, d), dtype=torch.bfloat16, device=DEV)
+    swa.decode(dims, o, q.to(DEV), k.to(DEV), v.to(DEV), kcd, vcd, dev_i32(pos), ws)
+    expect = oracle.decode(ref, q, k, v, pos, dims.scale)
+    assert_close(o.double().cpu().numpy(), expect, "decode bf16", bf16_out=True)
+
+
+def test_device_status_reports_bad_device_arguments():
+    dims = mk_dims(1, 4, 2, 64, 64)
+    kc, vc = swa.new_cache(dims, DEV)
+    k = torch.zeros(1, 8, 2, 64, dtype=torch.bfloat16, device=DEV)
+    swa.cache_append(dims, kc, vc, k, k, dev_i32([-5]), dev_i32([8]))
+    with pytest.raises(swa.SwaError) as e:
+        swa.device_status()
+    assert e.value.code == swa.SWA_ERR_DEVICE_ARG
+    swa.device_status()  # cleared
+    swa.cache_append(dims, kc, vc, k, k, dev_i32([0]), dev_i32([9]))  # n_tokens > max_tokens
+    with pytest.raises(swa.SwaError):
+        swa.device_status()
+    assert float(kc.abs().sum()) == 0.0
