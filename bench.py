@@ -273,10 +273,10 @@ class DecodeRun:
         q, k, v = self.inputs[self.i % len(self.inputs)]
         self.i += 1
         if events is not None:
-            events[0].record()
+            events[0][0].record()
         self.swa.decode(self.dims, self.out, q, k, v, self.kc, self.vc, self.pos, self.ws)
         if events is not None:
-            events[1].record()
+            events[0][1].record()
         self.pos.add_(1)
 
 

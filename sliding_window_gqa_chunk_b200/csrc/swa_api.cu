@@ -146,7 +146,15 @@ int encode_map(EncodeTiledFn fn, CUtensorMap* map, const void* ptr, int rank, co
   return SWA_OK;
 }
 
+// Progress words of trace builds (-DSWA_TRACE): host-mapped memory set by
+// swa_debug_set_trace; always NULL in normal builds.
+int* g_trace = nullptr;
+
 }  // namespace
+
+#ifdef SWA_TRACE
+extern "C" SWA_API void swa_debug_set_trace(void* host_mapped) { g_trace = static_cast<int*>(host_mapped); }
+#endif
 
 namespace swa {
 
@@ -260,6 +268,7 @@ int swa_prefill_chunk(const swa_dims* dims, void* out, const void* q, const void
   p.n_q_tiles = (max_tokens + 127) / 128;
   p.scale_log2 = dims->scale * 1.4426950408889634f;
   p.out_f32 = dims->out_dtype == SWA_DTYPE_F32;
+  p.trace = g_trace;
   cudaError_t e = swa::launch_prefill(p, maps, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "swa_prefill_chunk launch");
   return ok();

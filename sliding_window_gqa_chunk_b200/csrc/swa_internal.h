@@ -57,6 +57,7 @@ struct PrefillParams {
   int n_q_tiles;                // ceil(max_tokens / 128)
   float scale_log2;
   int out_f32;
+  int* trace;                   // progress words in host-mapped memory (trace builds only)
 };
 
 // TMA descriptors of the prefill, built on the host per call.

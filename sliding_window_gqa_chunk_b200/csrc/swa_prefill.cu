@@ -36,6 +36,23 @@ namespace swa {
 
 namespace {
 
+// Progress words for debugging hangs: compiled in only with -DSWA_TRACE, where
+// p.trace points at host-mapped memory the host can read while a kernel runs.
+#ifdef SWA_TRACE
+#define SWA_TRACE_AT(slot, value)                                                             \
+  do {                                                                                        \
+    if (p.trace != nullptr) {                                                                 \
+      const int cta_ = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;       \
+      *reinterpret_cast<volatile int*>(p.trace + cta_ * 8 + (slot)) = (value);                \
+      __threadfence_system();                                                                 \
+    }                                                                                         \
+  } while (0)
+#else
+#define SWA_TRACE_AT(slot, value) \
+  do {                            \
+  } while (0)
+#endif
+
 constexpr int kRows = 128;          // query rows per tile = TMEM lanes
 constexpr int kKeys = 128;          // keys per tile
 constexpr int kThreads = 320;       // 10 warps
@@ -201,14 +218,17 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
     tc::mbar_init(bar_done, 1);
     tc::mbar_fence_init();
   }
+  if (threadIdx.x == 0) SWA_TRACE_AT(0, 1);
   if (warp == kMmaWarp) {
     tc::tmem_alloc(tc::smem_u32(tmem_slot), kTmemCols);
     tc::tmem_relinquish();
+    if (lane == 0) SWA_TRACE_AT(0, 2);
   }
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) SWA_TRACE_AT(0, 3);
 
   if (warp == kProducerWarp) {
     // ============================ TMA producer ============================
@@ -226,8 +246,10 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
       bool ok = true;
       for (int j = 0; j < n_tiles && ok; ++j) {
         const int st = j % NS;
+        SWA_TRACE_AT(1, 1000 + j);
         if (j >= NS) ok = tc::mbar_wait(bar_kv_empty + 8 * st, ((j / NS) - 1) & 1, p.status);
         if (!ok) break;
+        SWA_TRACE_AT(1, 2000 + j);
         bool is_cache;
         int kbase;
         plan.at(j, is_cache, kbase);
@@ -253,12 +275,14 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
         }
       }
       // Before leaving, make sure no copy issued here is still in flight.
+      SWA_TRACE_AT(1, 5000);
       tc::mbar_wait(bar_q_full, 0, p.status);
       const int j0 = n_tiles > NS ? n_tiles - NS : 0;
       for (int j = j0; j < n_tiles; ++j) {
         tc::mbar_wait(bar_k_full + 8 * (j % NS), (j / NS) & 1, p.status);
         tc::mbar_wait(bar_v_full + 8 * (j % NS), (j / NS) & 1, p.status);
       }
+      SWA_TRACE_AT(1, 9999);
     }
   } else if (warp == kMmaWarp) {
     // ============================ MMA issuer ============================
@@ -288,10 +312,12 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
         }
       };
 
+      SWA_TRACE_AT(2, 10);
       bool ok = tc::mbar_wait(bar_q_full, 0, p.status);
       tc::tc_fence_after();
       for (int j = 0; j < n_tiles && ok; ++j) {
         const int st = j % NS;
+        SWA_TRACE_AT(2, 1000 + j);
         ok = tc::mbar_wait(bar_k_full + 8 * st, (j / NS) & 1, p.status);
         if (!ok) break;
         tc::tc_fence_after();
@@ -304,6 +330,7 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
             tc::tc_fence_after();
             issue_pv(i, sp, j - 1 > 0);
           }
+          SWA_TRACE_AT(2, 3000 + j * 2 + i);
           issue_s(i, st);
           tc::tc_commit(bar_s_full + 8 * i);
         }
@@ -317,13 +344,16 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
           if (ok && i == 0) ok = tc::mbar_wait(bar_v_full + 8 * sl, (jl / NS) & 1, p.status);
           if (!ok) break;
           tc::tc_fence_after();
+          SWA_TRACE_AT(2, 6000 + i);
           issue_pv(i, sl, jl > 0);
           tc::tc_commit(bar_o_full + 8 * i);
         }
       }
       // All MMAs must have finished before the TMEM is released.
+      SWA_TRACE_AT(2, 8000);
       tc::tc_commit(bar_done);
       tc::mbar_wait(bar_done, 0, p.status);
+      SWA_TRACE_AT(2, 9999);
     }
   } else if (warp / 4 < hpc) {
     // ============================ softmax / epilogue ============================
@@ -345,7 +375,10 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
     float l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      ok = tc::mbar_wait(bar_s_full + 8 * i, j & 1, p.status);
+      if (row == 0) SWA_TRACE_AT(3 + i, 1000 + j);
+      // tcgen05.ld / st / wait are warp-collective (.sync.aligned): every
+      // decision that guards them must be the same on all 32 lanes.
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_s_full + 8 * i, j & 1, p.status));
       if (!ok) break;
       tc::tc_fence_after();
       float sv[kKeys];
@@ -388,24 +421,30 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
 #pragma unroll
       for (int k = 1; k < kKeys; ++k) mx = fmaxf(mx, sv[k]);
       const float m_new = fmaxf(m_run, mx * sl2);
-      if (m_new > m_run + kRescaleThreshold) {
-        const float alpha = fast_exp2(m_run - m_new);  // 0 while nothing was visible yet
-        if (j > 0) {
-          // O_i holds the previous tiles' sum (its last PV finished before S_i(j) did)
-#pragma unroll
-          for (int c = 0; c < D / 16; ++c) {
-            float ov[16];
-            tc::tmem_ld16(tO + c * 16, ov);
-            tc::tc_wait_ld();
-            tc::reg_fence16(ov);
-            uint32_t ow[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) ow[e] = __float_as_uint(ov[e] * alpha);
-            tc::tmem_st16(tO + c * 16, ow);
-          }
-        }
+      // Rescale only when this row's max grew by more than 2^8; otherwise keep
+      // the stale max (p <= 2^8 stays exact enough in bf16 and fp32).
+      const bool grow = m_new > m_run + kRescaleThreshold;
+      float alpha = 1.f;
+      if (grow) {
+        alpha = fast_exp2(m_run - m_new);  // 0 while nothing was visible yet
         l_run *= alpha;
         m_run = m_new;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        // O_i holds the previous tiles' sum (its last PV finished before S_i(j)
+        // did).  The whole warp takes this branch; rows that keep their max
+        // multiply by 1.
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          float ov[16];
+          tc::tmem_ld16(tO + c * 16, ov);
+          tc::tc_wait_ld();
+          tc::reg_fence16(ov);
+          uint32_t ow[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) ow[e] = __float_as_uint(ov[e] * alpha);
+          tc::tmem_st16(tO + c * 16, ow);
+        }
       }
       const float nb = (m_run == -CUDART_INF_F) ? 0.f : -m_run;
 #pragma unroll
@@ -423,9 +462,12 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
       tc::tc_wait_st();
       tc::tc_fence_before();
       tc::mbar_arrive(bar_p_full + 8 * i);
+      if (row == 0) SWA_TRACE_AT(3 + i, 2000 + j);
     }
 
-    if (ok) ok = tc::mbar_wait(bar_o_full + 8 * i, 0, p.status);
+    if (row == 0) SWA_TRACE_AT(3 + i, 7000);
+    if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_o_full + 8 * i, 0, p.status));
+    if (row == 0) SWA_TRACE_AT(3 + i, ok ? 8000 : 7500);
     if (ok) {
       tc::tc_fence_after();
       const float inv_l = 1.f / l_run;
@@ -443,10 +485,13 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
   }
 
   tc::tc_fence_before();
+  if (threadIdx.x == 0) SWA_TRACE_AT(5, 1);
   __syncthreads();
+  if (threadIdx.x == 0) SWA_TRACE_AT(5, 2);
   if (warp == kMmaWarp) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, kTmemCols);
+    if (lane == 0) SWA_TRACE_AT(5, 3);
   }
 }
 
