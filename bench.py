@@ -166,6 +166,13 @@ def reduce_max(x: float, world: int) -> float:
     return float(t.item())
 
 
+def headline_config(wl, world: int) -> dict:
+    return {"workload": wl.name, "batch": 1, "seq_len": wl.lengths[0], "window": wl.shape.window,
+            "chunk": wl.chunk, "n_q_heads": 32, "n_kv_heads": 8, "head_dim": 128,
+            "out_dtype": "bf16", "l2": "flushed (256 MiB write) before every timed step",
+            "parallelism": f"replicas x{world}"}
+
+
 # ----------------------------------------------------------------------------
 # our implementation
 # ----------------------------------------------------------------------------
@@ -312,106 +319,120 @@ def bench_ours(args, world, rank, local):
     dev = f"cuda:{local}"
     peaks = load_peaks()
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    phase = args.phase
 
     def flush():
         flush_buf.fill_(1)
 
     wl = PREFILL_16K
-    run = PrefillRun(wl, "bf16", dev)
-    step = lambda ev: run.step(ev)  # noqa: E731
-
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        ms, per_call = time_steps(step, args.steps, args.warmup, flush, n_events=run.n_calls)
-    torch.cuda.synchronize()
-    barrier(world)
-    clocks = clk.summary()
-    ms_max = reduce_max(ms, world)
-    swa.device_status()
-
-    tokens = run.L
-    value = world * tokens / (ms_max / 1e3)
-    flops_step = sum(run.flops_per_call)
-    kernel_ms = sum(per_call)                   # prefill kernel time per step
-    avg_launch_ms = kernel_ms / run.n_calls
-    avg_flops = flops_step / run.n_calls
-    achieved_tflops = avg_flops / (avg_launch_ms / 1e3) / 1e12
-    peak = peaks["bf16_tflops"]
-
-    # decode phase
-    dec = DecodeRun(DECODE_B64, "bf16", dev)
-    dms, dpair = time_steps(lambda ev: dec.step(ev), args.steps, args.warmup, flush, n_events=1)
-    dms_max = reduce_max(dms, world)
-    dec_kernel_ms = dpair[0]
-    dec_gbs = dec.bytes_per_step / (dec_kernel_ms / 1e3) / 1e9
-    swa.device_status()
-
-    # dense causal comparator on the same inputs
-    dense_dims = swa.Dims(1, 32, 8, 128, 16384, wl.scale, "bf16")
-    dkc, dvc = swa.new_cache(dense_dims, dev)
-    zero = torch.zeros(1, dtype=torch.int32, device=dev)
-    full = torch.tensor([16384], dtype=torch.int32, device=dev)
-
-    def dense_step(ev):
-        if ev is not None:
-            ev[0][0].record()
-        swa.prefill_chunk(dense_dims, run.out, run.q, run.k, run.v, dkc, dvc, zero, full)
-        if ev is not None:
-            ev[0][1].record()
-
-    dense_ms, dense_pair = time_steps(dense_step, max(2, args.steps // 2), 2, flush, n_events=1)
-    dense_flops = 4.0 * 128 * 32 * prefill_pairs_per_head(16384, 16384, 16384)
-    swa.device_status()
-
-    # end to end through the public API with host buffers
-    e2e_ms, h2d, d2h = run_prefill_e2e(run, args.steps, min(args.warmup, 3), flush)
-    e2e_ms = reduce_max(e2e_ms, world)
-
     line = {
-        "metric": METRIC,
-        "value": round(value, 1),
-        "unit": "tokens/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
-        "ms_per_step": round(ms_max, 4),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "bf16",
-        "data": "synthetic",
-        "config": {"workload": wl.name, "batch": 1, "seq_len": run.L, "window": wl.shape.window,
-                   "chunk": wl.chunk, "n_q_heads": 32, "n_kv_heads": 8, "head_dim": 128,
-                   "out_dtype": "bf16", "l2": "flushed (256 MiB write) before every timed step",
-                   "parallelism": f"replicas x{world}"},
-        "tflops": round(flops_step / (ms_max / 1e3) / 1e12, 1),
-        "roofline": {"kernel": "swa_prefill_kernel", "bound": "tensor",
-                     "achieved": round(achieved_tflops, 1), "peak": peak,
-                     "unit": "TFLOP/s", "frac": round(achieved_tflops / peak, 4),
-                     "peak_source": f"{peaks['source']} bf16_tflops (burst)",
-                     "algorithmic_flops_per_launch": avg_flops, "traffic": None},
-        "decode": {"workload": DECODE_B64.name, "batch": DECODE_B64.batch,
-                   "tokens_per_s": round(world * DECODE_B64.batch / (dms_max / 1e3), 1),
-                   "ms_per_step": round(dms_max, 4),
-                   "roofline": {"kernel": "swa_decode_kernel+combine", "bound": "hbm",
-                                "achieved": round(dec_gbs, 1), "peak": peaks["hbm_gbs"],
-                                "unit": "GB/s", "frac": round(dec_gbs / peaks["hbm_gbs"], 4),
-                                "peak_source": f"{peaks['source']} hbm_gbs",
-                                "algorithmic_bytes_per_launch": dec.bytes_per_step,
-                                "traffic": None},
-                   "gpu_launches_per_step": dec.launches_per_step},
-        "dense": {"workload": "dense_causal_16k", "ms": round(dense_pair[0], 4),
-                  "tflops": round(dense_flops / (dense_pair[0] / 1e3) / 1e12, 1),
-                  "swa_speedup_vs_dense": round(dense_pair[0] / kernel_ms, 3)},
-        "e2e": {"value": round(world * tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": round(e2e_ms, 4)},
-        "gpu_launches": run.launches_per_step * args.steps,
-        "clocks": clocks,
+        "metric": METRIC, "value": None, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": headline_config(wl, world),
     }
-    if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
+    if phase != "all":
+        line["phase"] = phase
+
+    run = None
+    kernel_ms = None
+    if phase in ("all", "prefill", "dense"):
+        run = PrefillRun(wl, "bf16", dev)
+    if phase in ("all", "prefill"):
+        barrier(world)
+        torch.cuda.synchronize()
+        with ClockSampler(local) as clk:
+            ms, per_call = time_steps(lambda ev: run.step(ev), args.steps, args.warmup, flush,
+                                      n_events=run.n_calls)
+        torch.cuda.synchronize()
+        barrier(world)
+        ms_max = reduce_max(ms, world)
+        swa.device_status()
+        flops_step = sum(run.flops_per_call)
+        kernel_ms = sum(per_call)                   # prefill kernel time per step
+        avg_launch_ms = kernel_ms / run.n_calls
+        avg_flops = flops_step / run.n_calls
+        achieved = avg_flops / (avg_launch_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops"]
+        line.update({
+            "value": round(world * run.L / (ms_max / 1e3), 1),
+            "ms_per_step": round(ms_max, 4),
+            "tflops": round(flops_step / (ms_max / 1e3) / 1e12, 1),
+            "roofline": {"kernel": "swa_prefill_kernel", "bound": "tensor",
+                         "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(achieved / peak, 4),
+                         "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+                         "algorithmic_flops_per_launch": avg_flops,
+                         "launch_ms": [round(x, 4) for x in per_call], "traffic": None},
+            "gpu_launches": run.launches_per_step * args.steps,
+            "clocks": clk.summary(),
+        })
+
+    if phase in ("all", "decode"):
+        dec = DecodeRun(DECODE_B64, "bf16", dev)
+        barrier(world)
+        with ClockSampler(local) as dclk:
+            dms, dpair = time_steps(lambda ev: dec.step(ev), args.steps, args.warmup, flush,
+                                    n_events=1)
+        barrier(world)
+        dms_max = reduce_max(dms, world)
+        dec_kernel_ms = dpair[0]
+        dec_gbs = dec.bytes_per_step / (dec_kernel_ms / 1e3) / 1e9
+        swa.device_status()
+        dec_line = {
+            "workload": DECODE_B64.name, "batch": DECODE_B64.batch,
+            "tokens_per_s": round(world * DECODE_B64.batch / (dms_max / 1e3), 1),
+            "ms_per_step": round(dms_max, 4),
+            "roofline": {"kernel": "swa_decode_kernel (+ combine)", "bound": "hbm",
+                         "achieved": round(dec_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(dec_gbs / peaks["hbm_gbs"], 4),
+                         "peak_source": f"{peaks['source']} hbm_gbs",
+                         "algorithmic_bytes_per_launch": dec.bytes_per_step,
+                         "launch_ms": round(dec_kernel_ms, 4), "traffic": None},
+            "gpu_launches_per_step": dec.launches_per_step,
+            "clocks": dclk.summary(),
+        }
+        line["decode"] = dec_line
+        if phase == "decode":
+            line.update({"value": dec_line["tokens_per_s"], "ms_per_step": dec_line["ms_per_step"],
+                         "roofline": dec_line["roofline"], "clocks": dec_line["clocks"],
+                         "gpu_launches": dec.launches_per_step * args.steps})
+            line["config"] = {"workload": DECODE_B64.name, "batch": DECODE_B64.batch,
+                              "window": 4096, "n_q_heads": 32, "n_kv_heads": 8, "head_dim": 128,
+                              "out_dtype": "bf16", "l2": line["config"]["l2"],
+                              "parallelism": f"replicas x{world}"}
+
+    if phase in ("all", "dense"):
+        # dense causal comparator on the same inputs: one chunk of 16384, W = 16384
+        dense_dims = swa.Dims(1, 32, 8, 128, 16384, wl.scale, "bf16")
+        dkc, dvc = swa.new_cache(dense_dims, dev)
+        zero = torch.zeros(1, dtype=torch.int32, device=dev)
+        full = torch.tensor([16384], dtype=torch.int32, device=dev)
+
+        def dense_step(ev):
+            if ev is not None:
+                ev[0][0].record()
+            swa.prefill_chunk(dense_dims, run.out, run.q, run.k, run.v, dkc, dvc, zero, full)
+            if ev is not None:
+                ev[0][1].record()
+
+        _, dense_pair = time_steps(dense_step, max(2, args.steps // 2), 2, flush, n_events=1)
+        dense_flops = 4.0 * 128 * 32 * prefill_pairs_per_head(16384, 16384, 16384)
+        swa.device_status()
+        line["dense"] = {"workload": "dense_causal_16k", "ms": round(dense_pair[0], 4),
+                         "tflops": round(dense_flops / (dense_pair[0] / 1e3) / 1e12, 1)}
+        if kernel_ms:
+            line["dense"]["swa_speedup_vs_dense"] = round(dense_pair[0] / kernel_ms, 3)
+
+    if phase == "all":
+        # end to end through the public API with host buffers
+        e2e_ms, h2d, d2h = run_prefill_e2e(run, args.steps, 3, flush)
+        e2e_ms = reduce_max(e2e_ms, world)
+        line["e2e"] = {"value": round(world * run.L / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "ms_per_step": round(e2e_ms, 4)}
+        if rank == 0 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
     return line
 
 
@@ -470,9 +491,7 @@ def bench_reference(args, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(per * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "batch": 1, "seq_len": wl.lengths[0],
-                   "window": wl.shape.window, "chunk": wl.chunk, "n_q_heads": 32,
-                   "n_kv_heads": 8, "head_dim": 128, "parallelism": "cpu"},
+        "config": headline_config(wl, world),
         "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s",
                          "cores": oracle.max_threads(), "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -489,6 +508,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--ref-rows", type=int, default=128)
+    ap.add_argument("--phase", choices=["all", "prefill", "decode", "dense"], default="all",
+                    help="run one phase only (for profiling); the headline line needs 'all'")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
