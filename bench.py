@@ -43,6 +43,17 @@ from swa_workloads import (DECODE_B64, PREFILL_16K, decode_cache, decode_positio
                            decode_step_inputs, prefill_inputs)
 
 METRIC = ("prefill tokens/s & TFLOP/s (% bf16 peak); decode tokens/s & HBM GB/s (% peak)")
+
+# DRAM bytes (read + write) per launch from one ncu capture of each kernel, valid only
+# while the kernel source is the one that was profiled (sha256 prefix of the .cu file);
+# the summaries with the commands are under profiles/.
+PROFILED_TRAFFIC = {
+    "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "e51113a7ad1cfa27",
+                           "bytes": 67_200_512 + 8_282_624,
+                           "launch": "chunk 1 of 4 (every row sees 4096 keys)"},
+    "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "755fd51e78c93611",
+                          "bytes": 1_074_287_000 + 4_925_696, "launch": "one decode step"},
+}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 
@@ -164,6 +175,20 @@ def reduce_max(x: float, world: int) -> float:
     t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def profiled_traffic(kernel: str):
+    """ncu DRAM bytes per launch if the kernel source still matches the profiled one."""
+    import hashlib
+    rec = PROFILED_TRAFFIC[kernel]
+    path = os.path.join(ROOT, "sliding_window_gqa_chunk_b200", "csrc", rec["file"])
+    try:
+        sha = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None, None
+    if sha != rec["sha"]:
+        return None, None
+    return rec["bytes"], rec["launch"]
 
 
 def headline_config(wl, world: int) -> dict:
@@ -363,7 +388,9 @@ def bench_ours(args, world, rank, local):
                          "frac": round(achieved / peak, 4),
                          "peak_source": f"{peaks['source']} bf16_tflops (burst)",
                          "algorithmic_flops_per_launch": avg_flops,
-                         "launch_ms": [round(x, 4) for x in per_call], "traffic": None},
+                         "launch_ms": [round(x, 4) for x in per_call],
+                         "traffic": profiled_traffic("swa_prefill_kernel")[0],
+                         "traffic_launch": profiled_traffic("swa_prefill_kernel")[1]},
             "gpu_launches": run.launches_per_step * args.steps,
             "clocks": clk.summary(),
         })
@@ -388,7 +415,8 @@ def bench_ours(args, world, rank, local):
                          "frac": round(dec_gbs / peaks["hbm_gbs"], 4),
                          "peak_source": f"{peaks['source']} hbm_gbs",
                          "algorithmic_bytes_per_launch": dec.bytes_per_step,
-                         "launch_ms": round(dec_kernel_ms, 4), "traffic": None},
+                         "launch_ms": round(dec_kernel_ms, 4),
+                         "traffic": profiled_traffic("swa_decode_kernel")[0]},
             "gpu_launches_per_step": dec.launches_per_step,
             "clocks": dclk.summary(),
         }

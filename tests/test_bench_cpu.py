@@ -1,0 +1,93 @@
+"""Host-side logic of bench.py that needs no GPU: the algorithmic work counts,
+the max-over-ranks reduction (2 gloo ranks on CPU), the rank-0-only reference
+arm and the clock-sample parsing."""
+import json
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def test_pair_counts_match_the_closed_forms():
+    # SWA over 16384 tokens with W = 4096: W(W+1)/2 + (L - W) W pairs per head
+    assert bench.prefill_pairs_per_head(16384, 4096, 4096) == 4096 * 4097 // 2 + 12288 * 4096
+    assert bench.prefill_pairs_per_head(16384, 4096, 4096) == 58_722_304
+    # dense causal: L(L+1)/2
+    assert bench.prefill_pairs_per_head(16384, 16384, 16384) == 134_225_920
+    # per-chunk counts add up to the whole prompt
+    total = sum(bench.chunk_pairs_per_head(c * 4096, 4096, 4096) for c in range(4))
+    assert total == 58_722_304
+    flops = 4 * 128 * 32 * 58_722_304
+    assert abs(flops / 1e12 - 0.962) < 1e-3
+
+
+def test_decode_bytes_per_step():
+    from swa_workloads import DECODE_B64
+    B, W, Hkv, d, Hq = 64, 4096, 8, 128, 32
+    expect = B * (2 * W * Hkv * d * 2 + Hq * d * 2 + 2 * Hkv * d * 2 * 2 + Hq * d * 2)
+    assert expect == 1_075_314_688
+    assert DECODE_B64.batch == B and DECODE_B64.shape.window == W
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_main(rank, world, port, out_dir):
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port),
+                       "RANK": str(rank), "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank)})
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        bench.barrier(world)
+        got = bench.reduce_max(1.5 + rank * 2.25, world)
+        with open(os.path.join(out_dir, f"r{rank}.json"), "w") as f:
+            json.dump({"max": got}, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_reduce_max_over_two_gloo_ranks(tmp_path):
+    port = _free_port()
+    mp.start_processes(_rank_main, args=(2, port, str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+    for r in range(2):
+        with open(tmp_path / f"r{r}.json") as f:
+            assert json.load(f)["max"] == 3.75
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    class A:
+        steps, warmup, ref_rows = 1, 0, 4
+    assert bench.bench_reference(A, world=2, rank=1) is None
+    line = bench.bench_reference(A, world=1, rank=0)
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["config"] == bench.headline_config(bench.PREFILL_16K, 1)
+
+
+def test_clock_summary_parsing(tmp_path):
+    cs = bench.ClockSampler(0)
+    cs.path = str(tmp_path / "c.csv")
+    with open(cs.path, "w") as f:
+        f.write("0, 1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active\n")
+        f.write("0, 1800, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active\n")
+        f.write("0, 1700, 1965, 995.0, 0x4, Not Active, Not Active, Not Active, Active\n")
+    s = cs.summary()
+    assert s["sm_mhz"] == 1800 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_profiled_traffic_is_dropped_when_the_kernel_changes(monkeypatch):
+    rec = dict(bench.PROFILED_TRAFFIC["swa_decode_kernel"])
+    monkeypatch.setitem(bench.PROFILED_TRAFFIC, "swa_decode_kernel", dict(rec, sha="0" * 16))
+    assert bench.profiled_traffic("swa_decode_kernel") == (None, None)
