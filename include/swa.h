@@ -147,6 +147,32 @@ SWA_API int swa_decode(const swa_dims* dims, void* out, const void* q, const voi
                void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * swa_decode_static - swa_decode for callers that cannot allocate device
+ * memory.  The paper has no counterpart to this call; it exists for the
+ * library's users.  Some callers cannot allocate: an engine that plans all GPU
+ * memory up front and hands out only fixed buffers, or host code that gets
+ * tensor pointers from a framework that owns every allocation.  Such a caller
+ * passes the same inputs and outputs as to swa_decode (same meaning, layout
+ * and ownership) but no workspace.
+ *   - The decode scratch comes from one array built into the library,
+ *     4 MiB (4194304 bytes) per device, held by every GPU that loads the
+ *     library until the process exits.  Dims whose swa_decode_workspace_size
+ *     exceeds 4 MiB are rejected with SWA_ERR_WORKSPACE_TOO_SMALL and nothing
+ *     is enqueued.
+ *   - The call allocates nothing.  Its first call on each device looks up the
+ *     array's device address, with that device current; make that first call
+ *     before any stream capture begins.
+ *   - All calls on a device share the array, which keeps the previous call's
+ *     contents.  Nothing in it needs clearing, because each call writes every
+ *     scratch value it reads.  Calls that may overlap on the GPU (other
+ *     streams, unordered host threads) race on it: order them on one stream,
+ *     or use swa_decode with separate workspaces.
+ */
+SWA_API int swa_decode_static(const swa_dims* dims, void* out, const void* q, const void* k_new,
+                      const void* v_new, void* k_cache, void* v_cache, const int32_t* pos,
+                      void* stream);
+
+/*
  * swa_device_status - synchronise `stream`, then read and clear the library's
  * device status word on the current device: SWA_OK, SWA_ERR_TIMEOUT (a
  * bounded wait inside a kernel ran out; that kernel's outputs are invalid) or

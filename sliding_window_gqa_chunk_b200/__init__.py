@@ -35,7 +35,7 @@ import torch
 
 __all__ = [
     "Dims", "SwaError", "load_library", "library_path", "cache_append", "prefill_chunk",
-    "decode", "decode_workspace_size", "device_status", "new_cache", "abi_version",
+    "decode", "decode_static", "decode_workspace_size", "device_status", "new_cache", "abi_version",
     "SWA_OK", "SWA_ERR_INVALID_ARG", "SWA_ERR_UNSUPPORTED", "SWA_ERR_WORKSPACE_TOO_SMALL",
     "SWA_ERR_CUDA", "SWA_ERR_TIMEOUT", "SWA_ERR_DEVICE_ARG",
 ]
@@ -117,6 +117,8 @@ def load_library() -> ctypes.CDLL:
         lib.swa_decode_workspace_size.restype = ctypes.c_size_t
         lib.swa_decode.argtypes = [D, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         lib.swa_decode.restype = ctypes.c_int
+        lib.swa_decode_static.argtypes = [D, P, P, P, P, P, P, P, P]
+        lib.swa_decode_static.restype = ctypes.c_int
         lib.swa_device_status.argtypes = [P]
         lib.swa_device_status.restype = ctypes.c_int
         lib.swa_last_error.argtypes = []
@@ -190,6 +192,21 @@ def decode(dims: Dims, out, q, k_new, v_new, k_cache, v_cache, pos, workspace,
         ctypes.byref(cd), _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
         _ptr(v_cache), _ptr(pos), _ptr(workspace), int(workspace.numel() * workspace.element_size()),
         _stream(stream)))
+
+
+def decode_static(dims: Dims, out, q, k_new, v_new, k_cache, v_cache, pos, stream=None) -> None:
+    """swa_decode_static: the same decode step as ``decode`` with no workspace argument.
+
+    For callers that cannot allocate device memory (an engine with a fixed,
+    pre-planned arena, or code that only receives tensor pointers): the scratch
+    comes from a 4 MiB array built into the library, shared by every call on a
+    device.  Calls that may overlap on the GPU race on it; the first call on a
+    device should come before any stream capture.
+    """
+    cd = dims.c()
+    _check(load_library().swa_decode_static(
+        ctypes.byref(cd), _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+        _ptr(v_cache), _ptr(pos), _stream(stream)))
 
 
 def device_status(stream=None) -> None:

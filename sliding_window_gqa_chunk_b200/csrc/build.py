@@ -20,7 +20,7 @@ ROOT = os.path.dirname(PKG)
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libswa.so")
 
-SOURCES = ["swa_api.cu", "swa_append.cu", "swa_decode.cu", "swa_prefill.cu"]
+SOURCES = ["swa_api.cu", "swa_append.cu", "swa_decode.cu", "swa_prefill.cu", "swa_decode_static.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -342,3 +342,29 @@ int swa_device_status(void* stream) {
 }
 
 }  // extern "C"
+
+// Helpers for entry points defined in other translation units.
+namespace swa {
+
+int api_fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int api_ok() { return ok(); }
+
+int api_status_word(int** out) { return status_ptr(out); }
+
+int api_check_decode(const swa_dims* dims, const void* out, const void* q, const void* k_new,
+                     const void* v_new, const void* k_cache, const void* v_cache, const int32_t* pos) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_ptrs("out, q, k_new, v_new, k_cache, v_cache", {out, q, k_new, v_new, k_cache, v_cache})))
+    return rc;
+  return check_int_ptrs("pos", {pos});
+}
+
+}  // namespace swa

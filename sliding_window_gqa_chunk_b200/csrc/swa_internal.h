@@ -75,4 +75,13 @@ cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& maps, cuda
 // TMA box width (elements of d per box row) and swizzle span used by the prefill kernel.
 void prefill_map_geometry(int head_dim, int* box_elems, int* swizzle_bytes);
 
+// Helpers of the C-ABI layer for entry points defined in other files: set the
+// thread-local error message, look up the device status word, and run the
+// host-side argument checks of a decode call (everything but the workspace).
+int api_fail(int code, const char* fmt, ...);
+int api_ok();
+int api_status_word(int** out);
+int api_check_decode(const struct swa_dims* dims, const void* out, const void* q, const void* k_new,
+                     const void* v_new, const void* k_cache, const void* v_cache, const int32_t* pos);
+
 }  // namespace swa
