@@ -29,6 +29,7 @@
 #include <math_constants.h>
 
 #include "swa_common.cuh"
+#include "swa_exp2.cuh"
 #include "swa_internal.h"
 #include "swa_tc.cuh"
 
@@ -164,7 +165,9 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qt = blockIdx.x;
+  // Heaviest query tiles first: in a chunk that starts the prompt, tile qt has
+  // qt + 1 key tiles, so later tiles are dispatched first.
+  const int qt = gridDim.x - 1 - blockIdx.x;
   const int b = blockIdx.z;
   const int hpc = p.heads_per_cta;
   const int G = p.n_q_heads / p.n_kv_heads;
@@ -395,11 +398,12 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
       bool is_cache;
       int kbase;
       plan.at(j, is_cache, kbase);
+      bool masked = false;  // this row has invisible keys in this tile
       if (is_cache) {
         int d0 = kbase - a_i;
         if (d0 < 0) d0 += W;
-        const bool full = (kbase + kKeys <= W) && (len_i > 0) && (d0 + kKeys <= len_i);
-        if (!full) {
+        masked = !((kbase + kKeys <= W) && (len_i > 0) && (d0 + kKeys <= len_i));
+        if (masked) {
 #pragma unroll
           for (int k = 0; k < kKeys; ++k) {
             const int r = kbase + k;
@@ -410,16 +414,25 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
           }
         }
       } else {
-        if (kbase + kKeys - 1 > t) {
+        masked = kbase + kKeys - 1 > t;
+        if (masked) {
 #pragma unroll
           for (int k = 0; k < kKeys; ++k)
             if (kbase + k > t) sv[k] = -CUDART_INF_F;
         }
       }
 
-      float mx = sv[0];
+      // row maximum: 8 independent 3-input max chains, then a short tree
+      float mx8[8];
 #pragma unroll
-      for (int k = 1; k < kKeys; ++k) mx = fmaxf(mx, sv[k]);
+      for (int a = 0; a < 8; ++a) mx8[a] = fmaxf(sv[a], sv[8 + a]);
+#pragma unroll
+      for (int k = 16; k < kKeys; k += 16) {
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mx8[a] = fmax3(mx8[a], sv[k + a], sv[k + 8 + a]);
+      }
+      const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                             fmaxf(mx8[6], mx8[7]));
       const float m_new = fmaxf(m_run, mx * sl2);
       // Rescale only when this row's max grew by more than 2^8; otherwise keep
       // the stale max (p <= 2^8 stays exact enough in bf16 and fp32).
@@ -447,17 +460,36 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
         }
       }
       const float nb = (m_run == -CUDART_INF_F) ? 0.f : -m_run;
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      const uint64_t nbx2 = f2_pack(nb, nb);
+      uint64_t lsum[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+      // Tiles where some row masks keys take the SFU exp2 everywhere (exact 0
+      // for -inf); the others send 3 of every 8 pairs to the FMA pipe.
+      const bool sfu_only = __any_sync(0xffffffffu, masked);
 #pragma unroll
       for (int c = 0; c < kKeys / 32; ++c) {
         uint32_t pw[16];
 #pragma unroll
         for (int w = 0; w < 16; ++w) {
-          const float p0 = fast_exp2(fmaf(sv[c * 32 + 2 * w], sl2, nb));
-          const float p1 = fast_exp2(fmaf(sv[c * 32 + 2 * w + 1], sl2, nb));
-          l_run += p0 + p1;
+          const uint64_t x = f2_fma(f2_pack(sv[c * 32 + 2 * w], sv[c * 32 + 2 * w + 1]), sl2x2, nbx2);
+          float p0, p1;
+          f2_unpack(x, p0, p1);
+          if (!sfu_only && (w % 8 == 1 || w % 8 == 4 || w % 8 == 6)) {
+            exp2_fma_pipe(p0, p1);
+          } else {
+            p0 = fast_exp2(p0);
+            p1 = fast_exp2(p1);
+          }
+          lsum[w & 1] = f2_add(lsum[w & 1], f2_pack(p0, p1));
           pw[w] = pack_bf16x2(p0, p1);
         }
         tc::tmem_st16(tS + c * 16, pw);  // P (bf16 pairs) over the first 64 columns of S_i
+      }
+      {
+        float a0, a1, b0, b1;
+        f2_unpack(lsum[0], a0, a1);
+        f2_unpack(lsum[1], b0, b1);
+        l_run += (a0 + a1) + (b0 + b1);
       }
       tc::tc_wait_st();
       tc::tc_fence_before();
