@@ -6,7 +6,8 @@
 // head (GQA: both heads reuse every K/V tile the CTA loads).  Warp roles:
 //   warps 0-3  softmax for head slot 0 (TMEM lanes 0-127 = the 128 query rows)
 //   warps 4-7  softmax for head slot 1
-//   warp  8    TMA producer (Q once, then K/V tiles into an NS-stage ring)
+//   warp  8    TMA producer (Q once, then K tiles into an NK-stage ring and V
+//              tiles into an NV-stage ring)
 //   warp  9    TMEM allocator and the single thread issuing tcgen05.mma
 // Per key tile j and head slot i:
 //   S_i = Q_i K_j^T       tcgen05.mma, A = Q (smem), B = K (smem), D = S_i (TMEM, fp32)
@@ -62,6 +63,19 @@ constexpr int kMmaWarp = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
 constexpr uint32_t kTmemCols = 512;
 
+// Which of every 8 consecutive (even, odd) column pairs of a fully visible tile
+// take the FMA-pipe exp2 instead of the SFU (bit w set: pair w mod 8).
+#ifndef SWA_EXP2_FMA_PAIRS
+#define SWA_EXP2_FMA_PAIRS 0x00
+#endif
+// K / V ring depths for head_dim 128 (2 Q tiles + K + V must fit in 227 KB).
+#ifndef SWA_K_STAGES_D128
+#define SWA_K_STAGES_D128 3
+#endif
+#ifndef SWA_V_STAGES_D128
+#define SWA_V_STAGES_D128 2
+#endif
+
 template <int D>
 struct Cfg {
   static constexpr int kSwzBytes = (D * 2 >= 128) ? 128 : D * 2;  // swizzle span = bytes per box row
@@ -69,11 +83,14 @@ struct Cfg {
   static constexpr int kColBlocks = (D * 2) / kSwzBytes;          // boxes per 128-row tile
   static constexpr int kBlockBytes = kRows * kSwzBytes;           // one box
   static constexpr int kTileBytes = kRows * D * 2;                // one 128 x d bf16 tile
-  static constexpr int kStages = (D == 128) ? 2 : 4;
+  // K and V rings are separate: a K tile is released as soon as the S
+  // products of both heads have consumed it, a V tile after the PV products.
+  static constexpr int kKStages = (D == 128) ? SWA_K_STAGES_D128 : 4;
+  static constexpr int kVStages = (D == 128) ? SWA_V_STAGES_D128 : 4;
   static constexpr uint32_t kLayout = (kSwzBytes == 128) ? tc::kLayoutSW128 : tc::kLayoutSW32;
   static constexpr int kSBO = 8 * kSwzBytes;                       // stride of 8-row groups
   static constexpr int kKStepsPerBlock = kSwzBytes / 32;           // 16-element k-steps per box row
-  static constexpr int kSmemTiles = (2 + 2 * kStages) * kTileBytes;
+  static constexpr int kSmemTiles = (2 + kKStages + kVStages) * kTileBytes;
   static constexpr int kSmemBytes = kSmemTiles + 512 + 1024;       // barriers + alignment slack
   static_assert(kColBlocks * kSwzBytes == D * 2, "head_dim must fill whole swizzle rows");
 };
@@ -160,7 +177,8 @@ template <int D, typename OutT>
 __global__ void __launch_bounds__(kThreads, 1)
 swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps maps) {
   using C = Cfg<D>;
-  constexpr int NS = C::kStages;
+  constexpr int NK = C::kKStages;
+  constexpr int NV = C::kVStages;
   extern __shared__ uint8_t smem_raw[];
 
   const int warp = threadIdx.x >> 5;
@@ -192,15 +210,16 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
   uint8_t* base_ptr = smem_raw + (base - raw_addr);
   const uint32_t sQ = base;                                   // 2 tiles
-  const uint32_t sK = base + 2 * C::kTileBytes;               // NS tiles
-  const uint32_t sV = sK + NS * C::kTileBytes;                // NS tiles
+  const uint32_t sK = base + 2 * C::kTileBytes;               // NK tiles
+  const uint32_t sV = sK + NK * C::kTileBytes;                // NV tiles
   const uint32_t sBar = base + C::kSmemTiles;
   // barrier addresses (8 bytes each)
   const uint32_t bar_q_full = sBar;
-  const uint32_t bar_k_full = sBar + 8;                // [NS]
-  const uint32_t bar_v_full = bar_k_full + 8 * NS;     // [NS]
-  const uint32_t bar_kv_empty = bar_v_full + 8 * NS;   // [NS]
-  const uint32_t bar_s_full = bar_kv_empty + 8 * NS;   // [2]
+  const uint32_t bar_k_full = sBar + 8;                // [NK]
+  const uint32_t bar_k_empty = bar_k_full + 8 * NK;    // [NK]
+  const uint32_t bar_v_full = bar_k_empty + 8 * NK;    // [NV]
+  const uint32_t bar_v_empty = bar_v_full + 8 * NV;    // [NV]
+  const uint32_t bar_s_full = bar_v_empty + 8 * NV;    // [2]
   const uint32_t bar_p_full = bar_s_full + 16;         // [2]
   const uint32_t bar_o_full = bar_p_full + 16;         // [2]
   const uint32_t bar_done = bar_o_full + 16;
@@ -208,14 +227,17 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
 
   if (threadIdx.x == 0) {
     tc::mbar_init(bar_q_full, 1);
-    for (int i = 0; i < NS; ++i) {
+    for (int i = 0; i < NK; ++i) {
       tc::mbar_init(bar_k_full + 8 * i, 1);
+      tc::mbar_init(bar_k_empty + 8 * i, 1);
+    }
+    for (int i = 0; i < NV; ++i) {
       tc::mbar_init(bar_v_full + 8 * i, 1);
-      tc::mbar_init(bar_kv_empty + 8 * i, 1);
+      tc::mbar_init(bar_v_empty + 8 * i, 1);
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(bar_s_full + 8 * i, 1);
-      tc::mbar_init(bar_p_full + 8 * i, kRows);
+      tc::mbar_init(bar_p_full + 8 * i, kRows / 32);  // one arrival per softmax warp
       tc::mbar_init(bar_o_full + 8 * i, 1);
     }
     tc::mbar_init(bar_done, 1);
@@ -248,43 +270,44 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
                           h_first + i, t_lo, b, bar_q_full);
       bool ok = true;
       for (int j = 0; j < n_tiles && ok; ++j) {
-        const int st = j % NS;
-        SWA_TRACE_AT(1, 1000 + j);
-        if (j >= NS) ok = tc::mbar_wait(bar_kv_empty + 8 * st, ((j / NS) - 1) & 1, p.status);
-        if (!ok) break;
-        SWA_TRACE_AT(1, 2000 + j);
         bool is_cache;
         int kbase;
         plan.at(j, is_cache, kbase);
-        const uint32_t kdst = sK + st * C::kTileBytes;
-        const uint32_t vdst = sV + st * C::kTileBytes;
-        tc::mbar_arrive_expect_tx(bar_k_full + 8 * st, C::kTileBytes);
+        const int sk = j % NK, sv = j % NV;
+        SWA_TRACE_AT(1, 1000 + j);
+        if (j >= NK) ok = tc::mbar_wait(bar_k_empty + 8 * sk, ((j / NK) - 1) & 1, p.status);
+        if (!ok) break;
+        const uint32_t kdst = sK + sk * C::kTileBytes;
+        tc::mbar_arrive_expect_tx(bar_k_full + 8 * sk, C::kTileBytes);
         for (int cb = 0; cb < C::kColBlocks; ++cb) {
           if (is_cache)
             tc::tma_load_3d(kdst + cb * C::kBlockBytes, &maps.kc, cb * C::kBoxD, kbase,
-                            b * p.n_kv_heads + kvh, bar_k_full + 8 * st);
+                            b * p.n_kv_heads + kvh, bar_k_full + 8 * sk);
           else
             tc::tma_load_4d(kdst + cb * C::kBlockBytes, &maps.k, cb * C::kBoxD, kvh, kbase, b,
-                            bar_k_full + 8 * st);
+                            bar_k_full + 8 * sk);
         }
-        tc::mbar_arrive_expect_tx(bar_v_full + 8 * st, C::kTileBytes);
+        if (j >= NV) ok = tc::mbar_wait(bar_v_empty + 8 * sv, ((j / NV) - 1) & 1, p.status);
+        if (!ok) break;
+        SWA_TRACE_AT(1, 2000 + j);
+        const uint32_t vdst = sV + sv * C::kTileBytes;
+        tc::mbar_arrive_expect_tx(bar_v_full + 8 * sv, C::kTileBytes);
         for (int cb = 0; cb < C::kColBlocks; ++cb) {
           if (is_cache)
             tc::tma_load_3d(vdst + cb * C::kBlockBytes, &maps.vc, cb * C::kBoxD, kbase,
-                            b * p.n_kv_heads + kvh, bar_v_full + 8 * st);
+                            b * p.n_kv_heads + kvh, bar_v_full + 8 * sv);
           else
             tc::tma_load_4d(vdst + cb * C::kBlockBytes, &maps.v, cb * C::kBoxD, kvh, kbase, b,
-                            bar_v_full + 8 * st);
+                            bar_v_full + 8 * sv);
         }
       }
       // Before leaving, make sure no copy issued here is still in flight.
       SWA_TRACE_AT(1, 5000);
       tc::mbar_wait(bar_q_full, 0, p.status);
-      const int j0 = n_tiles > NS ? n_tiles - NS : 0;
-      for (int j = j0; j < n_tiles; ++j) {
-        tc::mbar_wait(bar_k_full + 8 * (j % NS), (j / NS) & 1, p.status);
-        tc::mbar_wait(bar_v_full + 8 * (j % NS), (j / NS) & 1, p.status);
-      }
+      for (int j = n_tiles > NK ? n_tiles - NK : 0; j < n_tiles; ++j)
+        tc::mbar_wait(bar_k_full + 8 * (j % NK), (j / NK) & 1, p.status);
+      for (int j = n_tiles > NV ? n_tiles - NV : 0; j < n_tiles; ++j)
+        tc::mbar_wait(bar_v_full + 8 * (j % NV), (j / NV) & 1, p.status);
       SWA_TRACE_AT(1, 9999);
     }
   } else if (warp == kMmaWarp) {
@@ -318,39 +341,37 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
       SWA_TRACE_AT(2, 10);
       bool ok = tc::mbar_wait(bar_q_full, 0, p.status);
       tc::tc_fence_after();
-      for (int j = 0; j < n_tiles && ok; ++j) {
-        const int st = j % NS;
-        SWA_TRACE_AT(2, 1000 + j);
-        ok = tc::mbar_wait(bar_k_full + 8 * st, (j / NS) & 1, p.status);
-        if (!ok) break;
-        tc::tc_fence_after();
+      // Per tile j: for each head slot i, O_i += P_i(j-1) V(j-1) (needs the
+      // softmax of tile j-1), then S_i(j) = Q_i K(j)^T.  A tcgen05.commit tracks
+      // every MMA issued before it, so the V stage is released right after the
+      // last PV that reads it and the K stage right after the last S.
+      for (int j = 0; j <= n_tiles && ok; ++j) {
+        const bool has_s = j < n_tiles;
+        const int sk = j % NK;
+        if (has_s) {
+          SWA_TRACE_AT(2, 1000 + j);
+          ok = tc::mbar_wait(bar_k_full + 8 * sk, (j / NK) & 1, p.status);
+          if (!ok) break;
+        }
+        const int svp = (j - 1) % NV;
         for (int i = 0; i < hpc && ok; ++i) {
           if (j > 0) {
-            const int sp = (j - 1) % NS;
             ok = tc::mbar_wait(bar_p_full + 8 * i, (j - 1) & 1, p.status);
-            if (ok && i == 0) ok = tc::mbar_wait(bar_v_full + 8 * sp, ((j - 1) / NS) & 1, p.status);
+            if (ok && i == 0) ok = tc::mbar_wait(bar_v_full + 8 * svp, ((j - 1) / NV) & 1, p.status);
             if (!ok) break;
             tc::tc_fence_after();
-            issue_pv(i, sp, j - 1 > 0);
+            issue_pv(i, svp, j - 1 > 0);
+            if (i == hpc - 1) tc::tc_commit(bar_v_empty + 8 * svp);
+            if (!has_s) tc::tc_commit(bar_o_full + 8 * i);
           }
-          SWA_TRACE_AT(2, 3000 + j * 2 + i);
-          issue_s(i, st);
-          tc::tc_commit(bar_s_full + 8 * i);
+          if (has_s) {
+            tc::tc_fence_after();
+            SWA_TRACE_AT(2, 3000 + j * 2 + i);
+            issue_s(i, sk);
+            tc::tc_commit(bar_s_full + 8 * i);
+          }
         }
-        if (ok && j > 0) tc::tc_commit(bar_kv_empty + 8 * ((j - 1) % NS));
-      }
-      if (ok) {
-        const int jl = n_tiles - 1;
-        const int sl = jl % NS;
-        for (int i = 0; i < hpc && ok; ++i) {
-          ok = tc::mbar_wait(bar_p_full + 8 * i, jl & 1, p.status);
-          if (ok && i == 0) ok = tc::mbar_wait(bar_v_full + 8 * sl, (jl / NS) & 1, p.status);
-          if (!ok) break;
-          tc::tc_fence_after();
-          SWA_TRACE_AT(2, 6000 + i);
-          issue_pv(i, sl, jl > 0);
-          tc::tc_commit(bar_o_full + 8 * i);
-        }
+        if (ok && has_s) tc::tc_commit(bar_k_empty + 8 * sk);
       }
       // All MMAs must have finished before the TMEM is released.
       SWA_TRACE_AT(2, 8000);
@@ -474,7 +495,7 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
           const uint64_t x = f2_fma(f2_pack(sv[c * 32 + 2 * w], sv[c * 32 + 2 * w + 1]), sl2x2, nbx2);
           float p0, p1;
           f2_unpack(x, p0, p1);
-          if (!sfu_only && (w % 8 == 1 || w % 8 == 4 || w % 8 == 6)) {
+          if (!sfu_only && ((SWA_EXP2_FMA_PAIRS >> (w % 8)) & 1)) {
             exp2_fma_pipe(p0, p1);
           } else {
             p0 = fast_exp2(p0);
@@ -493,7 +514,8 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
       }
       tc::tc_wait_st();
       tc::tc_fence_before();
-      tc::mbar_arrive(bar_p_full + 8 * i);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar_p_full + 8 * i);
       if (row == 0) SWA_TRACE_AT(3 + i, 2000 + j);
     }
 
