@@ -9,6 +9,10 @@
 //   warp  8    TMA producer (Q once, then K tiles into an NK-stage ring and V
 //              tiles into an NV-stage ring)
 //   warp  9    TMEM allocator and the single thread issuing tcgen05.mma
+//   warps 10-11 idle (they complete the third warpgroup)
+// The kernel is compiled for 168 registers per thread (12 warps); the third
+// warpgroup gives registers back (setmaxnreg) so that each softmax thread can
+// hold its whole 128-column row of S without spilling.
 // Per key tile j and head slot i:
 //   S_i = Q_i K_j^T       tcgen05.mma, A = Q (smem), B = K (smem), D = S_i (TMEM, fp32)
 //   softmax warps read S_i row by row (one thread per query row), mask, update
@@ -57,7 +61,16 @@ namespace {
 
 constexpr int kRows = 128;          // query rows per tile = TMEM lanes
 constexpr int kKeys = 128;          // keys per tile
-constexpr int kThreads = 320;       // 10 warps
+constexpr int kThreads = 384;       // 12 warps = 3 warpgroups
+// Register split: launched at kLaunchRegs per thread, the two softmax
+// warpgroups grow to kSoftmaxRegs and the producer/MMA warpgroup shrinks to
+// kOtherRegs.  2 * kSoftmaxRegs + kOtherRegs must equal 3 * kLaunchRegs (the
+// block's register pool), or setmaxnreg.inc would wait forever; the host
+// refuses to launch if ptxas did not allocate exactly kLaunchRegs.
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 224;
+constexpr int kOtherRegs = 56;
+static_assert(2 * kSoftmaxRegs + kOtherRegs == 3 * kLaunchRegs, "register split must fill the pool");
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
@@ -255,6 +268,10 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) SWA_TRACE_AT(0, 3);
 
+  // setmaxnreg is per warpgroup and must dominate the code it budgets, so the
+  // role dispatch happens inside the two register branches.
+  if (warp >= 8) {
+  tc::regs_decrease<kOtherRegs>();
   if (warp == kProducerWarp) {
     // ============================ TMA producer ============================
     if (lane == 0) {
@@ -379,7 +396,10 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
       tc::mbar_wait(bar_done, 0, p.status);
       SWA_TRACE_AT(2, 9999);
     }
-  } else if (warp / 4 < hpc) {
+  }
+  } else {
+  tc::regs_increase<kSoftmaxRegs>();
+  if (warp / 4 < hpc) {
     // ============================ softmax / epilogue ============================
     const int i = warp / 4;                   // head slot
     const int row = (warp % 4) * 32 + lane;   // query row within the tile = TMEM lane
@@ -537,6 +557,7 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
       }
     }
   }
+  }
 
   tc::tc_fence_before();
   if (threadIdx.x == 0) SWA_TRACE_AT(5, 1);
@@ -555,6 +576,15 @@ template <int D, typename OutT>
 cudaError_t launch_prefill_t(const PrefillParams& p, const PrefillMaps& maps, cudaStream_t stream) {
   using C = Cfg<D>;
   auto kern = swa_prefill_kernel<D, OutT>;
+  // The setmaxnreg split assumes the launch register count; never launch with another.
+  static int regs = -1;
+  if (regs < 0) {
+    cudaFuncAttributes attr;
+    cudaError_t ea = cudaFuncGetAttributes(&attr, kern);
+    if (ea != cudaSuccess) return ea;
+    regs = attr.numRegs;
+  }
+  if (regs != kLaunchRegs) return cudaErrorInvalidKernelImage;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(p.n_q_tiles, p.n_q_heads / p.heads_per_cta, p.batch);
