@@ -332,26 +332,32 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
     if (lane == 0) {
       constexpr uint32_t idesc_s = tc::make_idesc_bf16(kRows, kKeys, false, false);
       constexpr uint32_t idesc_pv = tc::make_idesc_bf16(kRows, D, false, true);
+      // Shared-memory descriptors are built once; a k-step or a stage only
+      // moves the start address, i.e. adds (bytes >> 4) to the low field
+      // (shared addresses stay below 2^18, so the 14-bit field never carries).
+      const uint64_t q_desc = tc::make_sdesc(sQ, 16, C::kSBO, C::kLayout);
+      const uint64_t k_desc = tc::make_sdesc(sK, 16, C::kSBO, C::kLayout);
+      const uint64_t v_desc = tc::make_sdesc(sV, C::kBlockBytes, C::kSBO, C::kLayout);
       auto issue_s = [&](int i, int st) {
         const uint32_t d_tmem = tmem + i * kKeys;
+        const uint64_t qd = q_desc + (uint64_t)((i * C::kTileBytes) >> 4);
+        const uint64_t kd = k_desc + (uint64_t)((st * C::kTileBytes) >> 4);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const int cb = ks / C::kKStepsPerBlock;
           const int kin = ks % C::kKStepsPerBlock;
-          const uint32_t off = cb * C::kBlockBytes + kin * 32;
-          const uint64_t ad = tc::make_sdesc(sQ + i * C::kTileBytes + off, 16, C::kSBO, C::kLayout);
-          const uint64_t bd = tc::make_sdesc(sK + st * C::kTileBytes + off, 16, C::kSBO, C::kLayout);
-          tc::mma_ss(d_tmem, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)((cb * C::kBlockBytes + kin * 32) >> 4);
+          tc::mma_ss(d_tmem, qd + off, kd + off, idesc_s, ks > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int i, int st, bool accumulate) {
         const uint32_t d_tmem = tmem + 2 * kKeys + i * D;
         const uint32_t a_tmem = tmem + i * kKeys;
+        const uint64_t vd = v_desc + (uint64_t)((st * C::kTileBytes) >> 4);
 #pragma unroll
         for (int ks = 0; ks < kKeys / 16; ++ks) {
-          const uint64_t bd = tc::make_sdesc(sV + st * C::kTileBytes + ks * 16 * C::kSwzBytes,
-                                             C::kBlockBytes, C::kSBO, C::kLayout);
-          tc::mma_ts(d_tmem, a_tmem + ks * 8, bd, idesc_pv, (accumulate || ks > 0) ? 1u : 0u);
+          const uint64_t off = (uint64_t)((ks * 16 * C::kSwzBytes) >> 4);
+          tc::mma_ts(d_tmem, a_tmem + ks * 8, vd + off, idesc_pv, (accumulate || ks > 0) ? 1u : 0u);
         }
       };
 
@@ -463,75 +469,97 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
         }
       }
 
-      // row maximum: 8 independent 3-input max chains, then a short tree
-      float mx8[8];
+      // P = exp2(scale * log2(e) * s - base) for the whole tile, written over
+      // the first 64 columns of S_i; returns this thread's sum of the fp32 p.
+      // With track_max it also returns the tile's largest raw score (the max
+      // chains run on the ALU pipe, beside the SFU exponentials).
+      auto exp_pass = [&](float base_neg, bool track_max, float& tile_max) -> float {
+        const uint64_t sl2x2 = f2_pack(sl2, sl2);
+        const uint64_t nbx2 = f2_pack(base_neg, base_neg);
+        uint64_t lsum[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+        float m8[8];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) mx8[a] = fmaxf(sv[a], sv[8 + a]);
+        for (int a = 0; a < 8; ++a) m8[a] = -CUDART_INF_F;
 #pragma unroll
-      for (int k = 16; k < kKeys; k += 16) {
+        for (int c = 0; c < kKeys / 32; ++c) {
+          uint32_t pw[16];
 #pragma unroll
-        for (int a = 0; a < 8; ++a) mx8[a] = fmax3(mx8[a], sv[k + a], sv[k + 8 + a]);
-      }
-      const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                             fmaxf(mx8[6], mx8[7]));
-      const float m_new = fmaxf(m_run, mx * sl2);
-      // Rescale only when this row's max grew by more than 2^8; otherwise keep
-      // the stale max (p <= 2^8 stays exact enough in bf16 and fp32).
-      const bool grow = m_new > m_run + kRescaleThreshold;
-      float alpha = 1.f;
-      if (grow) {
-        alpha = fast_exp2(m_run - m_new);  // 0 while nothing was visible yet
-        l_run *= alpha;
-        m_run = m_new;
-      }
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // O_i holds the previous tiles' sum (its last PV finished before S_i(j)
-        // did).  The whole warp takes this branch; rows that keep their max
-        // multiply by 1.
-#pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-          float ov[16];
-          tc::tmem_ld16(tO + c * 16, ov);
-          tc::tc_wait_ld();
-          tc::reg_fence16(ov);
-          uint32_t ow[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) ow[e] = __float_as_uint(ov[e] * alpha);
-          tc::tmem_st16(tO + c * 16, ow);
-        }
-      }
-      const float nb = (m_run == -CUDART_INF_F) ? 0.f : -m_run;
-      const uint64_t sl2x2 = f2_pack(sl2, sl2);
-      const uint64_t nbx2 = f2_pack(nb, nb);
-      uint64_t lsum[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-      // Tiles where some row masks keys take the SFU exp2 everywhere (exact 0
-      // for -inf); the others send 3 of every 8 pairs to the FMA pipe.
-      const bool sfu_only = __any_sync(0xffffffffu, masked);
-#pragma unroll
-      for (int c = 0; c < kKeys / 32; ++c) {
-        uint32_t pw[16];
-#pragma unroll
-        for (int w = 0; w < 16; ++w) {
-          const uint64_t x = f2_fma(f2_pack(sv[c * 32 + 2 * w], sv[c * 32 + 2 * w + 1]), sl2x2, nbx2);
-          float p0, p1;
-          f2_unpack(x, p0, p1);
-          if (!sfu_only && ((SWA_EXP2_FMA_PAIRS >> (w % 8)) & 1)) {
-            exp2_fma_pipe(p0, p1);
-          } else {
+          for (int w = 0; w < 16; ++w) {
+            const float s0 = sv[c * 32 + 2 * w], s1 = sv[c * 32 + 2 * w + 1];
+            if (track_max) m8[w % 8] = fmax3(m8[w % 8], s0, s1);
+            const uint64_t x = f2_fma(f2_pack(s0, s1), sl2x2, nbx2);
+            float p0, p1;
+            f2_unpack(x, p0, p1);
             p0 = fast_exp2(p0);
             p1 = fast_exp2(p1);
+            lsum[w & 1] = f2_add(lsum[w & 1], f2_pack(p0, p1));
+            pw[w] = pack_bf16x2(p0, p1);
           }
-          lsum[w & 1] = f2_add(lsum[w & 1], f2_pack(p0, p1));
-          pw[w] = pack_bf16x2(p0, p1);
+          tc::tmem_st16(tS + c * 16, pw);  // P (bf16 pairs) over the first 64 columns of S_i
         }
-        tc::tmem_st16(tS + c * 16, pw);  // P (bf16 pairs) over the first 64 columns of S_i
-      }
-      {
+        if (track_max)
+          tile_max = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
         float a0, a1, b0, b1;
         f2_unpack(lsum[0], a0, a1);
         f2_unpack(lsum[1], b0, b1);
-        l_run += (a0 + a1) + (b0 + b1);
+        return (a0 + a1) + (b0 + b1);
+      };
+
+      // Optimistic pass: exponentiate against the running max right away and
+      // check the tile's max afterwards.  Only if some row's max grew by more
+      // than 2^8 (always on a row's first visible tile) is the tile redone
+      // against the new max.  The decisions are warp-uniform because the
+      // TMEM accesses they guard are warp-collective.
+      float part = 0.f;
+      bool exact = __any_sync(0xffffffffu, m_run == -CUDART_INF_F);
+      if (!exact) {
+        float tmax;
+        part = exp_pass(-m_run, true, tmax);
+        exact = __any_sync(0xffffffffu, tmax * sl2 > m_run + kRescaleThreshold);
       }
+      if (exact) {
+        // row maximum: 8 independent 3-input max chains, then a short tree
+        float mx8[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mx8[a] = fmaxf(sv[a], sv[8 + a]);
+#pragma unroll
+        for (int k = 16; k < kKeys; k += 16) {
+#pragma unroll
+          for (int a = 0; a < 8; ++a) mx8[a] = fmax3(mx8[a], sv[k + a], sv[k + 8 + a]);
+        }
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                               fmaxf(mx8[6], mx8[7]));
+        const float m_new = fmaxf(m_run, mx * sl2);
+        // Rescale only when this row's max grew by more than 2^8; otherwise keep
+        // the stale max (p <= 2^8 stays exact enough in bf16 and fp32).
+        const bool grow = m_new > m_run + kRescaleThreshold;
+        float alpha = 1.f;
+        if (grow) {
+          alpha = fast_exp2(m_run - m_new);  // 0 while nothing was visible yet
+          l_run *= alpha;
+          m_run = m_new;
+        }
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          // O_i holds the previous tiles' sum (its last PV finished before S_i(j)
+          // did).  The whole warp takes this branch; rows that keep their max
+          // multiply by 1.
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) {
+            float ov[16];
+            tc::tmem_ld16(tO + c * 16, ov);
+            tc::tc_wait_ld();
+            tc::reg_fence16(ov);
+            uint32_t ow[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) ow[e] = __float_as_uint(ov[e] * alpha);
+            tc::tmem_st16(tO + c * 16, ow);
+          }
+        }
+        float unused;
+        part = exp_pass((m_run == -CUDART_INF_F) ? 0.f : -m_run, false, unused);
+      }
+      l_run += part;
+      (void)masked;
       tc::tc_wait_st();
       tc::tc_fence_before();
       __syncwarp();
