@@ -39,8 +39,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from swa_workloads import (DECODE_B64, PREFILL_16K, decode_cache, decode_positions,  # noqa: E402
-                           decode_step_inputs, prefill_inputs)
+from swa_workloads import (DECODE_B64, PREFILL_16K, decode_32l_workload, decode_cache,  # noqa: E402
+                           decode_positions, decode_step_inputs, prefill_inputs, varlen_workload)
 
 METRIC = ("prefill tokens/s & TFLOP/s (% bf16 peak); decode tokens/s & HBM GB/s (% peak)")
 
@@ -48,8 +48,8 @@ METRIC = ("prefill tokens/s & TFLOP/s (% bf16 peak); decode tokens/s & HBM GB/s 
 # while the kernel source is the one that was profiled (sha256 prefix of the .cu file);
 # the summaries with the commands are under profiles/.
 PROFILED_TRAFFIC = {
-    "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "e51113a7ad1cfa27",
-                           "bytes": 67_200_512 + 8_282_624,
+    "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "4a934635ab7980c7",
+                           "bytes": 67_203_840 + 5_355_264,
                            "launch": "chunk 1 of 4 (every row sees 4096 keys)"},
     "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "755fd51e78c93611",
                           "bytes": 1_074_287_000 + 4_925_696, "launch": "one decode step"},
@@ -85,63 +85,82 @@ def chunk_pairs_per_head(start: int, T: int, W: int) -> int:
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while active."""
+    """SM clock and throttle reasons sampled every millisecond (NVML) while active.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    The timed regions last milliseconds, far below nvidia-smi's sampling
+    period, so NVML is polled from a thread; nvidia-smi is the fallback.
+    """
 
-    def __init__(self, gpu_index: int):
+    NAMES = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+             ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4), ("hw_power_brake", 0x80))
+
+    def __init__(self, gpu_index: int, period_s: float = 0.001):
         self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+        self.period = period_s
+        self.samples = []
+        self.sm_max = None
+        self._stop = None
+        self._thread = None
+        self._nvml = None
 
     def __enter__(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
+        import threading
         try:
-            self.out = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=self.out, stderr=subprocess.DEVNULL)
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self._nvml = (pynvml, h)
+            self.sm_max = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
         except Exception:
-            self.proc = None
+            self._nvml = None
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                self._sample()
+                time.sleep(self.period)
+
+        self._sample()
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
         return self
 
-    def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
+    def _sample(self):
+        if self._nvml is not None:
+            pynvml, h = self._nvml
             try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-            self.out.close()
-
-    def summary(self):
-        rows = []
-        try:
-            with open(self.path) as f:
-                for line in f:
-                    parts = [p.strip() for p in line.split(",")]
-                    if len(parts) >= 9:
-                        rows.append(parts)
-        except Exception:
-            pass
-        finally:
-            try:
-                os.unlink(self.path)
+                sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                try:
+                    reasons = int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))
+                except Exception:
+                    reasons = int(pynvml.nvmlDeviceGetCurrentClocksThrottleReasons(h))
+                self.samples.append((sm, reasons))
             except Exception:
                 pass
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+            return
+        try:
+            out = subprocess.run(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=clocks.sm,clocks.max.sm",
+                 "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5).stdout
+            sm, mx = (float(x) for x in out.strip().split(","))
+            self.sm_max = mx
+            self.samples.append((sm, 0))
+        except Exception:
+            pass
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
+        self._sample()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.sm_max, "reasons": ["unsampled"]}
+        sms = [x[0] for x in self.samples]
+        reasons = sorted({name for _, r in self.samples for name, bit in self.NAMES if r & bit})
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": self.sm_max, "reasons": reasons,
+                "samples": len(self.samples), "source": "nvml" if self._nvml else "nvidia-smi"}
 
 
 def dist_setup(n_gpus: int):
@@ -312,6 +331,113 @@ class DecodeRun:
         self.pos.add_(1)
 
 
+class VarlenRun:
+    """Batched chunked prefill of 8 prompts (lengths uniform in [1024, 32768]).
+
+    Call c covers tokens [4096 c, 4096 (c + 1)) of every prompt still running;
+    the per-call inputs are laid out contiguously before timing."""
+
+    def __init__(self, wl, out_dtype="bf16", device="cuda"):
+        import sliding_window_gqa_chunk_b200 as swa
+        self.swa = swa
+        s = wl.shape
+        self.wl = wl
+        B, C = wl.batch, wl.chunk
+        self.dims = swa.Dims(B, s.n_q_heads, s.n_kv_heads, s.head_dim, s.window, wl.scale, out_dtype)
+        q, k, v = prefill_inputs(wl, device=device)
+        self.kc, self.vc = swa.new_cache(self.dims, device)
+        self.n_calls = (max(wl.lengths) + C - 1) // C
+        self.calls = []
+        flops = 0.0
+        for c in range(self.n_calls):
+            a = c * C
+            counts = [max(0, min(C, n - a)) for n in wl.lengths]
+            hi = min(q.shape[1], a + C)
+            def take(x):
+                buf = torch.zeros((B, C) + tuple(x.shape[2:]), dtype=x.dtype, device=device)
+                buf[:, : hi - a] = x[:, a:hi]
+                return buf
+            qc, kc, vc = take(q), take(k), take(v)
+            out = torch.empty((B, C, s.n_q_heads, s.head_dim), dtype=self.dims.torch_out_dtype,
+                              device=device)
+            sp = torch.tensor([a] * B, dtype=torch.int32, device=device)
+            nt = torch.tensor(counts, dtype=torch.int32, device=device)
+            self.calls.append((qc, kc, vc, out, sp, nt))
+            flops += sum(4.0 * s.head_dim * s.n_q_heads * chunk_pairs_per_head(a, n, s.window)
+                         for n in counts if n > 0)
+        del q, k, v
+        self.flops_per_step = flops
+        self.tokens = int(sum(wl.lengths))
+        self.launches_per_step = 2 * self.n_calls
+
+    def step(self, events=None):
+        for c, (qc, kc, vc, out, sp, nt) in enumerate(self.calls):
+            if events is not None:
+                events[c][0].record()
+            self.swa.prefill_chunk(self.dims, out, qc, kc, vc, self.kc, self.vc, sp, nt)
+            if events is not None:
+                events[c][1].record()
+            self.swa.cache_append(self.dims, self.kc, self.vc, kc, vc, sp, nt)
+
+
+class Decode32Run:
+    """One decode step through 32 layers (each with its own W = 4096 cache),
+    replayed as a CUDA graph of the 32 swa_decode calls."""
+
+    def __init__(self, wl, out_dtype="bf16", device="cuda"):
+        import sliding_window_gqa_chunk_b200 as swa
+        self.swa = swa
+        s = wl.shape
+        self.wl = wl
+        B = wl.batch
+        self.dims = swa.Dims(B, s.n_q_heads, s.n_kv_heads, s.head_dim, s.window, wl.scale, out_dtype)
+        g = torch.Generator(device=device)
+        g.manual_seed(wl.seed)
+        shape = (B, s.n_kv_heads, s.window, s.head_dim)
+        self.caches = []
+        for _ in range(wl.layers):
+            kc = torch.randn(shape, generator=g, device=device, dtype=torch.bfloat16)
+            vc = torch.randn(shape, generator=g, device=device, dtype=torch.bfloat16)
+            self.caches.append((kc, vc))
+        self.q = torch.randn((B, s.n_q_heads, s.head_dim), generator=g, device=device, dtype=torch.bfloat16)
+        self.k = torch.randn((B, s.n_kv_heads, s.head_dim), generator=g, device=device, dtype=torch.bfloat16)
+        self.v = torch.randn((B, s.n_kv_heads, s.head_dim), generator=g, device=device, dtype=torch.bfloat16)
+        self.out = torch.empty((B, s.n_q_heads, s.head_dim), dtype=self.dims.torch_out_dtype, device=device)
+        self.pos = decode_positions(wl, device=device)
+        self.ws = torch.empty(max(16, swa.decode_workspace_size(self.dims)), dtype=torch.uint8, device=device)
+        out_b = 4 if out_dtype == "f32" else 2
+        per_layer = B * (2 * s.window * s.n_kv_heads * s.head_dim * 2 + s.n_q_heads * s.head_dim * 2 +
+                         2 * s.n_kv_heads * s.head_dim * 2 * 2 + s.n_q_heads * s.head_dim * out_b)
+        self.bytes_per_step = wl.layers * per_layer
+        self.graph = None
+        per_call = 1 if swa.decode_workspace_size(self.dims) <= 16 else 2
+        self.launches_per_step = wl.layers * per_call + 1
+
+    def _layers(self):
+        for kc, vc in self.caches:
+            self.swa.decode(self.dims, self.out, self.q, self.k, self.v, kc, vc, self.pos, self.ws)
+        self.pos.add_(1)
+
+    def capture(self):
+        self._layers()                       # first calls on the device happen outside capture
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self._layers()
+        torch.cuda.synchronize()
+
+    def step(self, events=None):
+        if events is not None:
+            events[0][0].record()
+        self.graph.replay()
+        if events is not None:
+            events[0][1].record()
+
+    def release(self):
+        self.graph = None
+        self.caches = None
+
+
 def time_steps(fn, steps, warmup, flush, n_events=1):
     """Per-step CUDA-event timing with an L2 flush before every step (outside the
     timed interval).  Returns (mean step ms, mean per-event-pair ms list)."""
@@ -452,6 +578,48 @@ def bench_ours(args, world, rank, local):
         if kernel_ms:
             line["dense"]["swa_speedup_vs_dense"] = round(dense_pair[0] / kernel_ms, 3)
 
+    if phase in ("all", "varlen"):
+        vr = VarlenRun(varlen_workload(), "bf16", dev)
+        barrier(world)
+        vms, vpair = time_steps(lambda ev: vr.step(ev), max(3, args.steps // 2), 2, flush,
+                                n_events=vr.n_calls)
+        vms_max = reduce_max(vms, world)
+        swa.device_status()
+        vk = sum(vpair)
+        line["varlen"] = {
+            "workload": vr.wl.name, "lengths": list(vr.wl.lengths),
+            "tokens_per_s": round(world * vr.tokens / (vms_max / 1e3), 1),
+            "ms_per_step": round(vms_max, 4),
+            "tflops": round(vr.flops_per_step / (vms_max / 1e3) / 1e12, 1),
+            "roofline": {"kernel": "swa_prefill_kernel", "bound": "tensor",
+                         "achieved": round(vr.flops_per_step / (vk / 1e3) / 1e12, 1),
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": round(vr.flops_per_step / (vk / 1e3) / 1e12 / peaks["bf16_tflops"], 4)},
+            "gpu_launches_per_step": vr.launches_per_step}
+        del vr
+        torch.cuda.empty_cache()
+
+    if phase in ("all", "decode32"):
+        rows = []
+        for B in (1, 16, 64, 128):
+            dr = Decode32Run(decode_32l_workload(B), "bf16", dev)
+            dr.capture()
+            barrier(world)
+            dms32, dpair32 = time_steps(lambda ev: dr.step(ev), args.steps, args.warmup, flush,
+                                        n_events=1)
+            dms32 = reduce_max(dms32, world)
+            swa.device_status()
+            gbs = dr.bytes_per_step / (dpair32[0] / 1e3) / 1e9
+            rows.append({"batch": B, "tokens_per_s": round(world * B / (dms32 / 1e3), 1),
+                         "ms_per_step": round(dms32, 4),
+                         "hbm_gbs": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4),
+                         "gpu_launches_per_step": dr.launches_per_step})
+            dr.release()
+            del dr
+            torch.cuda.empty_cache()
+        line["decode_32layer"] = {"workload": "decode_32layer_w4096 (CUDA graph of 32 layer calls)",
+                                  "roofline_peak_gbs": peaks["hbm_gbs"], "rows": rows}
+
     if phase == "all":
         # end to end through the public API with host buffers
         e2e_ms, h2d, d2h = run_prefill_e2e(run, args.steps, 3, flush)
@@ -536,7 +704,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--ref-rows", type=int, default=128)
-    ap.add_argument("--phase", choices=["all", "prefill", "decode", "dense"], default="all",
+    ap.add_argument("--phase", choices=["all", "prefill", "decode", "dense", "varlen", "decode32"],
+                    default="all",
                     help="run one phase only (for profiling); the headline line needs 'all'")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":

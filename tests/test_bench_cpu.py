@@ -75,16 +75,15 @@ def test_reference_arm_runs_on_rank_zero_only():
     assert line["config"] == bench.headline_config(bench.PREFILL_16K, 1)
 
 
-def test_clock_summary_parsing(tmp_path):
+def test_clock_summary_reports_median_and_reasons():
     cs = bench.ClockSampler(0)
-    cs.path = str(tmp_path / "c.csv")
-    with open(cs.path, "w") as f:
-        f.write("0, 1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active\n")
-        f.write("0, 1800, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active\n")
-        f.write("0, 1700, 1965, 995.0, 0x4, Not Active, Not Active, Not Active, Active\n")
+    cs.sm_max = 1965.0
+    cs.samples = [(1965.0, 0x0), (1800.0, 0x4), (1700.0, 0x4)]
     s = cs.summary()
     assert s["sm_mhz"] == 1800 and s["sm_max_mhz"] == 1965
     assert s["reasons"] == ["sw_power_cap"]
+    cs.samples.append((1500.0, 0x40))
+    assert "hw_thermal_slowdown" in cs.summary()["reasons"]
 
 
 def test_profiled_traffic_is_dropped_when_the_kernel_changes(monkeypatch):
