@@ -17,10 +17,9 @@
 //   2^n by adding n to the exponent field (an integer multiply-add of the
 //   rounding sum's bit pattern by 2^23).
 //
-// Inputs must be finite and at most +128; they are clamped below at -126 so
-// the result stays a normal float (2^-126 instead of 0 for very negative
-// arguments, negligible next to the row's maximum term 1).  Masked entries
-// (-inf) must take the SFU path, which returns an exact 0.
+// Inputs must be at most +128.  Arguments below -126 (masked keys are -inf)
+// give exactly 0, so a masked key contributes nothing, as on the SFU path;
+// the polynomial itself only ever sees arguments in [-126, 128].
 #pragma once
 
 #include <stdint.h>
@@ -81,8 +80,11 @@ __device__ __forceinline__ void exp2_fma_pipe(float& x0, float& x1) {
   f2_unpack(j, j0, j1);
   // bits(2^n * p) = bits(p) + n * 2^23; the low bits of bits(j) are n (mod 2^9
   // after the shift), and unsigned arithmetic wraps as the two's complement needs.
-  x0 = __uint_as_float(__float_as_uint(j0) * (1u << 23) + __float_as_uint(p0));
-  x1 = __uint_as_float(__float_as_uint(j1) * (1u << 23) + __float_as_uint(p1));
+  const float y0 = __uint_as_float(__float_as_uint(j0) * (1u << 23) + __float_as_uint(p0));
+  const float y1 = __uint_as_float(__float_as_uint(j1) * (1u << 23) + __float_as_uint(p1));
+  // below the clamp (masked keys are -inf) the result is exactly 0
+  x0 = x0 >= -126.f ? y0 : 0.f;
+  x1 = x1 >= -126.f ? y1 : 0.f;
 }
 
 }  // namespace swa

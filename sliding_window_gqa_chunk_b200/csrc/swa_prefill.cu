@@ -6,10 +6,10 @@
 // head (GQA: both heads reuse every K/V tile the CTA loads).  Warp roles:
 //   warps 0-3  softmax for head slot 0 (TMEM lanes 0-127 = the 128 query rows)
 //   warps 4-7  softmax for head slot 1
-//   warp  8    TMA producer (Q once, then K tiles into an NK-stage ring and V
-//              tiles into an NV-stage ring)
-//   warp  9    TMEM allocator and the single thread issuing tcgen05.mma
-//   warps 10-11 idle (they complete the third warpgroup)
+//   warp  8    TMA producer: Q once, then K tiles into an NK-stage ring
+//   warp  9    TMEM allocator and MMA issuer (one elected lane issues tcgen05.mma)
+//   warp 10    TMA producer: V tiles into an NV-stage ring
+//   warp 11    idle (it completes the third warpgroup)
 // The kernel is compiled for 168 registers per thread (12 warps); the third
 // warpgroup gives registers back (setmaxnreg) so that each softmax thread can
 // hold its whole 128-column row of S without spilling.
@@ -73,8 +73,17 @@ constexpr int kOtherRegs = 56;
 static_assert(2 * kSoftmaxRegs + kOtherRegs == 3 * kLaunchRegs, "register split must fill the pool");
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kVProducerWarp = 10;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
 constexpr uint32_t kTmemCols = 512;
+// Which of every 8 consecutive (even, odd) column pairs take the FMA-pipe
+// exp2 (swa_exp2.cuh) instead of the SFU: bit w set means pair w mod 8.  The
+// SFU's exp2 has a quarter of the FMA pipe's lane rate, so moving a fraction
+// of the pairs shortens the softmax pass.  Both paths give exactly 0 for a
+// masked key (-inf).
+#ifndef SWA_EXP2_FMA_PAIRS
+#define SWA_EXP2_FMA_PAIRS 0x00
+#endif
 
 // Which of every 8 consecutive (even, odd) column pairs of a fully visible tile
 // take the FMA-pipe exp2 instead of the SFU (bit w set: pair w mod 8).
@@ -273,13 +282,11 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
   if (warp >= 8) {
   tc::regs_decrease<kOtherRegs>();
   if (warp == kProducerWarp) {
-    // ============================ TMA producer ============================
+    // ====================== TMA producer: Q, then K tiles ======================
     if (lane == 0) {
       tc::prefetch_map(&maps.q);
       tc::prefetch_map(&maps.k);
-      tc::prefetch_map(&maps.v);
       tc::prefetch_map(&maps.kc);
-      tc::prefetch_map(&maps.vc);
       tc::mbar_arrive_expect_tx(bar_q_full, hpc * C::kTileBytes);
       for (int i = 0; i < hpc; ++i)
         for (int cb = 0; cb < C::kColBlocks; ++cb)
@@ -290,7 +297,7 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
         bool is_cache;
         int kbase;
         plan.at(j, is_cache, kbase);
-        const int sk = j % NK, sv = j % NV;
+        const int sk = j % NK;
         SWA_TRACE_AT(1, 1000 + j);
         if (j >= NK) ok = tc::mbar_wait(bar_k_empty + 8 * sk, ((j / NK) - 1) & 1, p.status);
         if (!ok) break;
@@ -304,9 +311,29 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
             tc::tma_load_4d(kdst + cb * C::kBlockBytes, &maps.k, cb * C::kBoxD, kvh, kbase, b,
                             bar_k_full + 8 * sk);
         }
+      }
+      // Before leaving, make sure no copy issued here is still in flight.
+      SWA_TRACE_AT(1, 5000);
+      tc::mbar_wait(bar_q_full, 0, p.status);
+      for (int j = n_tiles > NK ? n_tiles - NK : 0; j < n_tiles; ++j)
+        tc::mbar_wait(bar_k_full + 8 * (j % NK), (j / NK) & 1, p.status);
+      SWA_TRACE_AT(1, 9999);
+    }
+  } else if (warp == kVProducerWarp) {
+    // ========================= TMA producer: V tiles =========================
+    // A separate issuer, so that a K load never waits behind a V stage that is
+    // still being read (the V ring turns over one iteration later than K's).
+    if (lane == 0) {
+      tc::prefetch_map(&maps.v);
+      tc::prefetch_map(&maps.vc);
+      bool ok = true;
+      for (int j = 0; j < n_tiles && ok; ++j) {
+        bool is_cache;
+        int kbase;
+        plan.at(j, is_cache, kbase);
+        const int sv = j % NV;
         if (j >= NV) ok = tc::mbar_wait(bar_v_empty + 8 * sv, ((j / NV) - 1) & 1, p.status);
         if (!ok) break;
-        SWA_TRACE_AT(1, 2000 + j);
         const uint32_t vdst = sV + sv * C::kTileBytes;
         tc::mbar_arrive_expect_tx(bar_v_full + 8 * sv, C::kTileBytes);
         for (int cb = 0; cb < C::kColBlocks; ++cb) {
@@ -318,18 +345,14 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
                             bar_v_full + 8 * sv);
         }
       }
-      // Before leaving, make sure no copy issued here is still in flight.
-      SWA_TRACE_AT(1, 5000);
-      tc::mbar_wait(bar_q_full, 0, p.status);
-      for (int j = n_tiles > NK ? n_tiles - NK : 0; j < n_tiles; ++j)
-        tc::mbar_wait(bar_k_full + 8 * (j % NK), (j / NK) & 1, p.status);
       for (int j = n_tiles > NV ? n_tiles - NV : 0; j < n_tiles; ++j)
         tc::mbar_wait(bar_v_full + 8 * (j % NV), (j / NV) & 1, p.status);
-      SWA_TRACE_AT(1, 9999);
     }
   } else if (warp == kMmaWarp) {
     // ============================ MMA issuer ============================
-    if (lane == 0) {
+    // The whole warp runs this loop converged (warp-uniform waits); one
+    // elected lane issues each tcgen05.mma / commit.
+    {
       constexpr uint32_t idesc_s = tc::make_idesc_bf16(kRows, kKeys, false, false);
       constexpr uint32_t idesc_pv = tc::make_idesc_bf16(kRows, D, false, true);
       // Shared-memory descriptors are built once; a k-step or a stage only
@@ -347,7 +370,7 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
           const int cb = ks / C::kKStepsPerBlock;
           const int kin = ks % C::kKStepsPerBlock;
           const uint64_t off = (uint64_t)((cb * C::kBlockBytes + kin * 32) >> 4);
-          tc::mma_ss(d_tmem, qd + off, kd + off, idesc_s, ks > 0 ? 1u : 0u);
+          tc::mma_ss_elect(d_tmem, qd + off, kd + off, idesc_s, ks > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int i, int st, bool accumulate) {
@@ -357,12 +380,12 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
 #pragma unroll
         for (int ks = 0; ks < kKeys / 16; ++ks) {
           const uint64_t off = (uint64_t)((ks * 16 * C::kSwzBytes) >> 4);
-          tc::mma_ts(d_tmem, a_tmem + ks * 8, vd + off, idesc_pv, (accumulate || ks > 0) ? 1u : 0u);
+          tc::mma_ts_elect(d_tmem, a_tmem + ks * 8, vd + off, idesc_pv, (accumulate || ks > 0) ? 1u : 0u);
         }
       };
 
       SWA_TRACE_AT(2, 10);
-      bool ok = tc::mbar_wait(bar_q_full, 0, p.status);
+      bool ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_q_full, 0, p.status));
       tc::tc_fence_after();
       // Per tile j: for each head slot i, O_i += P_i(j-1) V(j-1) (needs the
       // softmax of tile j-1), then S_i(j) = Q_i K(j)^T.  A tcgen05.commit tracks
@@ -373,32 +396,32 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
         const int sk = j % NK;
         if (has_s) {
           SWA_TRACE_AT(2, 1000 + j);
-          ok = tc::mbar_wait(bar_k_full + 8 * sk, (j / NK) & 1, p.status);
+          ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_k_full + 8 * sk, (j / NK) & 1, p.status));
           if (!ok) break;
         }
         const int svp = (j - 1) % NV;
         for (int i = 0; i < hpc && ok; ++i) {
           if (j > 0) {
-            ok = tc::mbar_wait(bar_p_full + 8 * i, (j - 1) & 1, p.status);
-            if (ok && i == 0) ok = tc::mbar_wait(bar_v_full + 8 * svp, ((j - 1) / NV) & 1, p.status);
+            ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_p_full + 8 * i, (j - 1) & 1, p.status));
+            if (ok && i == 0) ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_v_full + 8 * svp, ((j - 1) / NV) & 1, p.status));
             if (!ok) break;
             tc::tc_fence_after();
             issue_pv(i, svp, j - 1 > 0);
-            if (i == hpc - 1) tc::tc_commit(bar_v_empty + 8 * svp);
-            if (!has_s) tc::tc_commit(bar_o_full + 8 * i);
+            if (i == hpc - 1) tc::tc_commit_elect(bar_v_empty + 8 * svp);
+            if (!has_s) tc::tc_commit_elect(bar_o_full + 8 * i);
           }
           if (has_s) {
             tc::tc_fence_after();
             SWA_TRACE_AT(2, 3000 + j * 2 + i);
             issue_s(i, sk);
-            tc::tc_commit(bar_s_full + 8 * i);
+            tc::tc_commit_elect(bar_s_full + 8 * i);
           }
         }
-        if (ok && has_s) tc::tc_commit(bar_k_empty + 8 * sk);
+        if (ok && has_s) tc::tc_commit_elect(bar_k_empty + 8 * sk);
       }
       // All MMAs must have finished before the TMEM is released.
       SWA_TRACE_AT(2, 8000);
-      tc::tc_commit(bar_done);
+      tc::tc_commit_elect(bar_done);
       tc::mbar_wait(bar_done, 0, p.status);
       SWA_TRACE_AT(2, 9999);
     }
@@ -451,12 +474,13 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
         if (d0 < 0) d0 += W;
         masked = !((kbase + kKeys <= W) && (len_i > 0) && (d0 + kKeys <= len_i));
         if (masked) {
+          // slot kbase + k is visible iff it is < W and (kbase + k - a_i) mod W
+          // < len_i, i.e. k < len_i - d0, or W - d0 <= k < W - d0 + len_i
+          const int a_end = len_i - d0, b_lo = W - d0, b_end = W - d0 + len_i;
+          const int r_end = W - kbase;
 #pragma unroll
           for (int k = 0; k < kKeys; ++k) {
-            const int r = kbase + k;
-            int dd = r - a_i;
-            if (dd < 0) dd += W;
-            const bool vis = (r < W) && (dd < len_i);
+            const bool vis = (k < a_end || (k >= b_lo && k < b_end)) && k < r_end;
             if (!vis) sv[k] = -CUDART_INF_F;
           }
         }
@@ -490,8 +514,12 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
             const uint64_t x = f2_fma(f2_pack(s0, s1), sl2x2, nbx2);
             float p0, p1;
             f2_unpack(x, p0, p1);
-            p0 = fast_exp2(p0);
-            p1 = fast_exp2(p1);
+            if ((SWA_EXP2_FMA_PAIRS >> (w % 8)) & 1) {
+              exp2_fma_pipe(p0, p1);
+            } else {
+              p0 = fast_exp2(p0);
+              p1 = fast_exp2(p1);
+            }
             lsum[w & 1] = f2_add(lsum[w & 1], f2_pack(p0, p1));
             pw[w] = pack_bf16x2(p0, p1);
           }

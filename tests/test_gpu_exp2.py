@@ -52,3 +52,18 @@ def test_fma_pipe_exp2_error_bound():
     np.testing.assert_array_equal(fma_pipe[ints], exact[ints])
     # the SFU path stays within its own documented few-ulp error
     assert (np.abs(sfu - exact) / exact).max() < 1e-6
+
+
+def test_fma_pipe_exp2_is_exactly_zero_for_masked_keys():
+    # A masked key enters the softmax as -inf; it must contribute exactly 0,
+    # as the SFU's exp2(-inf) does.  So must anything below the clamp.
+    lib = _lib()
+    x = torch.tensor([-float("inf"), -1e30, -200.0, -126.5, -127.0, -126.0, 0.0, 1.0])
+    xd = x.cuda()
+    outs = [torch.empty_like(xd) for _ in range(3)]
+    assert lib.exp2_check(xd.data_ptr(), outs[0].data_ptr(), outs[1].data_ptr(),
+                          outs[2].data_ptr(), xd.numel()) == 0
+    got = outs[0].cpu().numpy()
+    assert (got[:5] == 0.0).all(), got
+    assert got[5] == 2.0 ** -126 and got[6] == 1.0 and got[7] == 2.0
+    assert (outs[1].cpu().numpy()[:1] == 0.0).all()
