@@ -294,6 +294,16 @@ def run_prefill_e2e(run: PrefillRun, steps: int, warmup: int, flush):
     return sum(times) / len(times), h2d, d2h
 
 
+def decode_launches_per_call(dims, swa_mod):
+    """Kernels one swa_decode call launches.  Few (sequence, kv head) pairs
+    (batch x n_kv_heads < 64) run as one launch whose splits merge inside a
+    thread-block cluster; otherwise a split sweep is followed by a combine
+    kernel whenever the workspace holds per-split partials."""
+    if dims.batch * dims.n_kv_heads < 64:
+        return 1
+    return 1 if swa_mod.decode_workspace_size(dims) <= 16 else 2
+
+
 class DecodeRun:
     """One decode step of batch 64 (positions uniform in [4096, 32768))."""
 
@@ -318,7 +328,7 @@ class DecodeRun:
         # q, the new k/v (read once, written once into the cache), the output
         self.bytes_per_step = B * (2 * W * Hkv * d * 2 + Hq * d * 2 + 2 * Hkv * d * 2 * 2 +
                                    Hq * d * out_b)
-        self.launches_per_step = 1 if swa.decode_workspace_size(self.dims) <= 16 else 2
+        self.launches_per_step = decode_launches_per_call(self.dims, swa)
 
     def step(self, events=None):
         q, k, v = self.inputs[self.i % len(self.inputs)]
@@ -410,8 +420,7 @@ class Decode32Run:
                          2 * s.n_kv_heads * s.head_dim * 2 * 2 + s.n_q_heads * s.head_dim * out_b)
         self.bytes_per_step = wl.layers * per_layer
         self.graph = None
-        per_call = 1 if swa.decode_workspace_size(self.dims) <= 16 else 2
-        self.launches_per_step = wl.layers * per_call + 1
+        self.launches_per_step = wl.layers * decode_launches_per_call(self.dims, swa) + 1
 
     def _layers(self):
         for kc, vc in self.caches:

@@ -158,10 +158,11 @@ extern "C" SWA_API void swa_debug_set_trace(void* host_mapped) { g_trace = stati
 
 namespace swa {
 
-DecodeSplit decode_split(int batch, int n_kv_heads, int window) {
-  // Aim for about four resident 128-thread CTAs per SM on a 148-SM B200; each
-  // split is a multiple of 64 slots (16 per warp).
+DecodeSplit decode_split(int batch, int n_q_heads, int n_kv_heads, int window) {
   const long long units = (long long)batch * n_kv_heads;
+  // Workspace split: about four resident 128-thread CTAs per SM on a 148-SM
+  // B200, each split a multiple of 64 slots (16 per warp); the per-split fp32
+  // partials are merged by a second kernel.
   const long long target = 148LL * 4;
   long long splits = (target + units - 1) / units;
   const long long max_splits = (window + 63) / 64;
@@ -172,6 +173,25 @@ DecodeSplit decode_split(int batch, int n_kv_heads, int window) {
   DecodeSplit s;
   s.slots_per_split = (int)per;
   s.n_splits = (int)((window + per - 1) / per);
+  s.ws_splits = s.n_splits;
+  s.warps = 4;
+  s.cluster = 0;
+  if (units < 64) {
+    // Few (sequence, kv head) pairs: the sweep is latency-bound, so each pair
+    // gets one cluster of up to 8 CTAs of 16 warps (8 for groups above 8
+    // heads, which need more registers), at least one 16-slot block per
+    // warp, merged in distributed shared memory: one launch, no workspace.
+    const int warps = (n_kv_heads > 0 && n_q_heads / n_kv_heads > 8) ? 8 : 16;
+    long long cs = (window + 16LL * warps - 1) / (16LL * warps);
+    if (cs > 8) cs = 8;
+    if (cs < 1) cs = 1;
+    long long cper = (window + cs - 1) / cs;
+    cper = (cper + 15) / 16 * 16;
+    s.slots_per_split = (int)cper;
+    s.n_splits = (int)((window + cper - 1) / cper);
+    s.warps = warps;
+    s.cluster = s.n_splits > 1 ? 1 : 0;
+  }
   return s;
 }
 
@@ -276,9 +296,10 @@ int swa_prefill_chunk(const swa_dims* dims, void* out, const void* q, const void
 
 size_t swa_decode_workspace_size(const swa_dims* dims) {
   if (check_dims(dims) != SWA_OK) return 0;
-  const swa::DecodeSplit sp = swa::decode_split(dims->batch, dims->n_kv_heads, dims->window);
-  if (sp.n_splits <= 1) return 16;  // nothing needed; a non-zero size keeps callers simple
-  const size_t bh = (size_t)dims->batch * dims->n_q_heads * sp.n_splits;
+  const swa::DecodeSplit sp =
+      swa::decode_split(dims->batch, dims->n_q_heads, dims->n_kv_heads, dims->window);
+  if (sp.ws_splits <= 1) return 16;  // nothing needed; a non-zero size keeps callers simple
+  const size_t bh = (size_t)dims->batch * dims->n_q_heads * sp.ws_splits;
   return bh * dims->head_dim * sizeof(float) + bh * 2 * sizeof(float);
 }
 
@@ -296,7 +317,8 @@ int swa_decode(const swa_dims* dims, void* out, const void* q, const void* k_new
     return fail(SWA_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
   int* status = nullptr;
   if ((rc = status_ptr(&status))) return rc;
-  const swa::DecodeSplit sp = swa::decode_split(dims->batch, dims->n_kv_heads, dims->window);
+  const swa::DecodeSplit sp =
+      swa::decode_split(dims->batch, dims->n_q_heads, dims->n_kv_heads, dims->window);
   swa::DecodeParams p;
   p.out = out;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -307,7 +329,7 @@ int swa_decode(const swa_dims* dims, void* out, const void* q, const void* k_new
   p.k_cache_w = static_cast<__nv_bfloat16*>(k_cache);
   p.v_cache_w = static_cast<__nv_bfloat16*>(v_cache);
   p.pos = pos;
-  const size_t bh = (size_t)dims->batch * dims->n_q_heads * sp.n_splits;
+  const size_t bh = (size_t)dims->batch * dims->n_q_heads * sp.ws_splits;
   p.ws_o = static_cast<float*>(workspace);
   p.ws_ml = static_cast<float*>(workspace) + bh * dims->head_dim;
   p.status = status;
@@ -318,6 +340,8 @@ int swa_decode(const swa_dims* dims, void* out, const void* q, const void* k_new
   p.window = dims->window;
   p.n_splits = sp.n_splits;
   p.slots_per_split = sp.slots_per_split;
+  p.warps = sp.warps;
+  p.cluster = sp.cluster;
   p.scale_log2 = dims->scale * 1.4426950408889634f;
   p.out_f32 = dims->out_dtype == SWA_DTYPE_F32;
   cudaError_t e = swa::launch_decode(p, static_cast<cudaStream_t>(stream));

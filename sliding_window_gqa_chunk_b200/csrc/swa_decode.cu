@@ -21,13 +21,18 @@
 // byte permutes.  P^T goes from the S accumulator layout to the B-operand
 // layout with one movmatrix.trans per 8x8 block.
 //
-// Work split: grid (n_splits, Hkv, B); a CTA of 4 warps covers one split of
-// the W slots; warps take interleaved 16-slot blocks, merge their (m, l, O)
-// in shared memory, and write either the final output (one split) or an fp32
-// partial for swa_decode_combine_kernel.  The CTA whose split holds slot
+// Work split: grid (n_splits, Hkv, B); a CTA of NW warps covers one split of
+// the W slots; warps take interleaved 16-slot blocks and merge their (m, l, O)
+// in shared memory.  Then the CTA writes the final output (one split), or the
+// splits of a (sequence, kv head) merge their partials: through distributed
+// shared memory when they form a thread-block cluster (few sequences, where
+// the sweep is latency-bound and a second launch would cost as much as the
+// sweep), else as fp32 partials in the workspace for
+// swa_decode_combine_kernel.  The CTA whose split holds slot
 // pos mod W writes the new key/value there; every lane that would read that
 // slot reads k_new / v_new instead, so no CTA ever reads a slot that is being
 // written.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -38,7 +43,6 @@ namespace swa {
 
 namespace {
 
-constexpr int kDecodeWarps = 4;
 constexpr int kBlockSlots = 16;
 
 // Physical element offset (within a row) of lane-quad t's key piece `j`
@@ -121,8 +125,8 @@ __device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* dst, flo
 }  // namespace
 
 // NT = number of 8-head n-tiles (ceil(G / 8)).
-template <int D, int NT, typename OutT>
-__global__ void __launch_bounds__(kDecodeWarps * 32)
+template <int D, int NT, int NW, typename OutT>
+__global__ void __launch_bounds__(NW * 32)
 swa_decode_kernel(const DecodeParams p) {
   using F = Frag<D>;
   extern __shared__ float smem[];
@@ -189,7 +193,7 @@ swa_decode_kernel(const DecodeParams p) {
   }
   const float sl2 = p.scale_log2;
 
-  for (int blk = r_begin + warp * kBlockSlots; blk < r_end; blk += kDecodeWarps * kBlockSlots) {
+  for (int blk = r_begin + warp * kBlockSlots; blk < r_end; blk += NW * kBlockSlots) {
     // ---- loads: K rows blk+g, blk+8+g; V rows blk+2t, +1, +8, +9 ----
     uint32_t kw0[F::kKWords], kw1[F::kKWords];
     {
@@ -268,12 +272,16 @@ swa_decode_kernel(const DecodeParams p) {
     }
   }
 
-  // ---- merge the 4 warps of the CTA ----
-  // smem: m[4][G8], l[4][G8], O[4][G8][D] with G8 = 8*NT
+  // ---- merge the NW warps of the CTA ----
+  // smem: m[NW][G8], l[NW][G8], O[NW][G8][D] with G8 = 8*NT, then the CTA's
+  // partial m[G8], l[G8], O[G8][D] (cluster merge)
   constexpr int G8 = 8 * NT;
   float* sm_m = smem;
-  float* sm_l = sm_m + kDecodeWarps * G8;
-  float* sm_o = sm_l + kDecodeWarps * G8;
+  float* sm_l = sm_m + NW * G8;
+  float* sm_o = sm_l + NW * G8;
+  float* cta_m = sm_o + (size_t)NW * G8 * D;
+  float* cta_l = cta_m + G8;
+  float* cta_o = cta_l + G8;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     float l0 = l_run[nt][0], l1 = l_run[nt][1];
@@ -314,11 +322,11 @@ swa_decode_kernel(const DecodeParams p) {
     const int dd = idx - h * D;
     float M = -CUDART_INF_F;
 #pragma unroll
-    for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, sm_m[w * G8 + h]);
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, sm_m[w * G8 + h]);
     float L = 0.f, O = 0.f;
     if (M != -CUDART_INF_F) {
 #pragma unroll
-      for (int w = 0; w < kDecodeWarps; ++w) {
+      for (int w = 0; w < NW; ++w) {
         const float sc = fast_exp2(sm_m[w * G8 + h] - M);
         L += sc * sm_l[w * G8 + h];
         O += sc * sm_o[((size_t)w * G8 + h) * D + dd];
@@ -327,6 +335,12 @@ swa_decode_kernel(const DecodeParams p) {
     const size_t bh = (size_t)b * p.n_q_heads + hq0 + h;
     if (p.n_splits == 1) {
       store_out<OutT>(reinterpret_cast<OutT*>(p.out) + bh * D + dd, O / L);
+    } else if (p.cluster) {
+      cta_o[h * D + dd] = O;
+      if (dd == 0) {
+        cta_m[h] = M;
+        cta_l[h] = L;
+      }
     } else {
       p.ws_o[(bh * p.n_splits + split) * D + dd] = O;
       if (dd == 0) {
@@ -334,6 +348,37 @@ swa_decode_kernel(const DecodeParams p) {
         p.ws_ml[(bh * p.n_splits + split) * 2 + 1] = L;
       }
     }
+  }
+
+  if (p.cluster) {
+    // The n_splits CTAs of this (sequence, kv head) are one cluster: each
+    // merges a share of the G x d outputs from every CTA's partial, read
+    // through distributed shared memory.  Every CTA of the cluster reaches
+    // both barriers (no CTA of a cluster returns early: they share pos).
+    namespace cg = cooperative_groups;
+    cg::cluster_group cl = cg::this_cluster();
+    cl.sync();
+    const int rank = (int)cl.block_rank();
+    const int R = p.n_splits;
+    for (int idx = rank * blockDim.x + threadIdx.x; idx < G * D; idx += R * blockDim.x) {
+      const int h = idx / D;
+      const int dd = idx - h * D;
+      float M = -CUDART_INF_F;
+      for (int r = 0; r < R; ++r) M = fmaxf(M, cl.map_shared_rank(cta_m, r)[h]);
+      float L = 0.f, O = 0.f;
+      if (M != -CUDART_INF_F) {
+        for (int r = 0; r < R; ++r) {
+          const float m = cl.map_shared_rank(cta_m, r)[h];
+          if (m == -CUDART_INF_F) continue;
+          const float sc = fast_exp2(m - M);
+          L += sc * cl.map_shared_rank(cta_l, r)[h];
+          O += sc * cl.map_shared_rank(cta_o, r)[h * D + dd];
+        }
+      }
+      const size_t bh = (size_t)b * p.n_q_heads + hq0 + h;
+      store_out<OutT>(reinterpret_cast<OutT*>(p.out) + bh * D + dd, O / L);
+    }
+    cl.sync();  // keep this CTA's partial alive until every peer has read it
   }
 }
 
@@ -362,17 +407,32 @@ swa_decode_combine_kernel(const DecodeParams p) {
 
 namespace {
 
-template <int D, int NT, typename OutT>
+template <int D, int NT, int NW, typename OutT>
 cudaError_t launch_decode_t(const DecodeParams& p, cudaStream_t stream) {
   constexpr int G8 = 8 * NT;
-  const size_t smem = sizeof(float) * (size_t)kDecodeWarps * G8 * (2 + D);
-  auto kern = swa_decode_kernel<D, NT, OutT>;
+  const size_t smem = sizeof(float) * (size_t)(NW + 1) * G8 * (2 + D);
+  auto kern = swa_decode_kernel<D, NT, NW, OutT>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
   dim3 grid(p.n_splits, p.n_kv_heads, p.batch);
-  kern<<<grid, kDecodeWarps * 32, smem, stream>>>(p);
+  if (p.cluster) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(NW * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)p.n_splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p);
+  }
+  kern<<<grid, NW * 32, smem, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || p.n_splits == 1) return e;
   swa_decode_combine_kernel<D, OutT><<<(unsigned)((size_t)p.batch * p.n_q_heads), D < 32 ? 32 : D, 0,
@@ -383,8 +443,12 @@ cudaError_t launch_decode_t(const DecodeParams& p, cudaStream_t stream) {
 template <int D, typename OutT>
 cudaError_t launch_decode_d(const DecodeParams& p, cudaStream_t stream) {
   const int G = p.n_q_heads / p.n_kv_heads;
-  if (G <= 8) return launch_decode_t<D, 1, OutT>(p, stream);
-  return launch_decode_t<D, 2, OutT>(p, stream);
+  if (G <= 8) {
+    if (p.warps == 16) return launch_decode_t<D, 1, 16, OutT>(p, stream);
+    return launch_decode_t<D, 1, 4, OutT>(p, stream);
+  }
+  if (p.warps == 8) return launch_decode_t<D, 2, 8, OutT>(p, stream);
+  return launch_decode_t<D, 2, 4, OutT>(p, stream);
 }
 
 template <typename OutT>

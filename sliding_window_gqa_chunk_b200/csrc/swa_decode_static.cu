@@ -87,7 +87,8 @@ extern "C" SWA_API int swa_decode_static(const swa_dims* dims, void* out, const 
   int* status = nullptr;
   if ((rc = swa::api_status_word(&status))) return rc;
 
-  const swa::DecodeSplit sp = swa::decode_split(dims->batch, dims->n_kv_heads, dims->window);
+  const swa::DecodeSplit sp =
+      swa::decode_split(dims->batch, dims->n_q_heads, dims->n_kv_heads, dims->window);
   swa::DecodeParams p;
   p.out = out;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -98,7 +99,7 @@ extern "C" SWA_API int swa_decode_static(const swa_dims* dims, void* out, const 
   p.k_cache_w = static_cast<__nv_bfloat16*>(k_cache);
   p.v_cache_w = static_cast<__nv_bfloat16*>(v_cache);
   p.pos = pos;
-  const size_t bh = (size_t)dims->batch * dims->n_q_heads * sp.n_splits;
+  const size_t bh = (size_t)dims->batch * dims->n_q_heads * sp.ws_splits;
   p.ws_o = static_cast<float*>(scratch);
   p.ws_ml = static_cast<float*>(scratch) + bh * dims->head_dim;
   p.status = status;
@@ -109,6 +110,8 @@ extern "C" SWA_API int swa_decode_static(const swa_dims* dims, void* out, const 
   p.window = dims->window;
   p.n_splits = sp.n_splits;
   p.slots_per_split = sp.slots_per_split;
+  p.warps = sp.warps;
+  p.cluster = sp.cluster;
   p.scale_log2 = dims->scale * 1.4426950408889634f;
   p.out_f32 = dims->out_dtype == SWA_DTYPE_F32;
   cudaError_t e = swa::launch_decode(p, static_cast<cudaStream_t>(stream));

@@ -35,6 +35,10 @@ struct DecodeParams {
   int* status;
   int batch, n_q_heads, n_kv_heads, head_dim, window;
   int n_splits, slots_per_split;
+  int warps;                    // warps per CTA
+  int cluster;                  // 1: the n_splits CTAs of a (sequence, kv head) form a
+                                // thread-block cluster and merge through distributed
+                                // shared memory (no workspace, no combine kernel)
   float scale_log2;             // scale * log2(e)
   int out_f32;
 };
@@ -44,8 +48,11 @@ struct DecodeParams {
 struct DecodeSplit {
   int n_splits;
   int slots_per_split;
+  int warps;
+  int cluster;
+  int ws_splits;   // splits the workspace is sized for (fp32 partials per split)
 };
-DecodeSplit decode_split(int batch, int n_kv_heads, int window);
+DecodeSplit decode_split(int batch, int n_q_heads, int n_kv_heads, int window);
 
 struct PrefillParams {
   void* out;                    // [B][max_tokens][Hq][d] bf16 or f32

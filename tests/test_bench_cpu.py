@@ -90,3 +90,13 @@ def test_profiled_traffic_is_dropped_when_the_kernel_changes(monkeypatch):
     rec = dict(bench.PROFILED_TRAFFIC["swa_decode_kernel"])
     monkeypatch.setitem(bench.PROFILED_TRAFFIC, "swa_decode_kernel", dict(rec, sha="0" * 16))
     assert bench.profiled_traffic("swa_decode_kernel") == (None, None)
+
+
+def test_decode_launch_count_follows_the_split_rule():
+    import sliding_window_gqa_chunk_b200 as swa
+    mk = lambda B: swa.Dims(B, 32, 8, 128, 4096, 1.0 / 128 ** 0.5, "bf16")
+    # batch 1 and 4: one launch (clustered splits); 64: sweep + combine; 128: one split
+    assert bench.decode_launches_per_call(mk(1), swa) == 1
+    assert bench.decode_launches_per_call(mk(4), swa) == 1
+    assert bench.decode_launches_per_call(mk(64), swa) == 2
+    assert bench.decode_launches_per_call(mk(128), swa) == 1
