@@ -158,6 +158,16 @@ extern "C" SWA_API void swa_debug_set_trace(void* host_mapped) { g_trace = stati
 
 namespace swa {
 
+// Largest thread-block cluster of the decode's split merge (8 is the portable
+// limit; 16 needs the non-portable opt-in, set at launch).
+#ifndef SWA_DECODE_MAX_CLUSTER
+#define SWA_DECODE_MAX_CLUSTER 8
+#endif
+// 0: never merge splits in a cluster (always the workspace and the combine kernel)
+#ifndef SWA_DECODE_CLUSTER
+#define SWA_DECODE_CLUSTER 1
+#endif
+
 DecodeSplit decode_split(int batch, int n_q_heads, int n_kv_heads, int window) {
   const long long units = (long long)batch * n_kv_heads;
   // Workspace split: about four resident 128-thread CTAs per SM on a 148-SM
@@ -176,14 +186,14 @@ DecodeSplit decode_split(int batch, int n_q_heads, int n_kv_heads, int window) {
   s.ws_splits = s.n_splits;
   s.warps = 4;
   s.cluster = 0;
-  if (units < 64) {
+  if (SWA_DECODE_CLUSTER && units < 64) {
     // Few (sequence, kv head) pairs: the sweep is latency-bound, so each pair
     // gets one cluster of up to 8 CTAs of 16 warps (8 for groups above 8
     // heads, which need more registers), at least one 16-slot block per
     // warp, merged in distributed shared memory: one launch, no workspace.
     const int warps = (n_kv_heads > 0 && n_q_heads / n_kv_heads > 8) ? 8 : 16;
     long long cs = (window + 16LL * warps - 1) / (16LL * warps);
-    if (cs > 8) cs = 8;
+    if (cs > SWA_DECODE_MAX_CLUSTER) cs = SWA_DECODE_MAX_CLUSTER;
     if (cs < 1) cs = 1;
     long long cper = (window + cs - 1) / cs;
     cper = (cper + 15) / 16 * 16;

@@ -113,6 +113,14 @@ __device__ __forceinline__ void load_v_row(uint32_t (&w)[Frag<D>::kVWords], cons
   }
 }
 
+// Programmatic dependent launch: the kernels below are launched with
+// programmatic stream serialization, so they may be scheduled while the
+// previous kernel in the stream is still running; this wait (first thing in
+// each kernel) returns once that kernel has completed and its memory writes
+// are visible, which keeps ordinary stream order for everything they read or
+// write.  Only the launch latency is overlapped.
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 template <typename OutT>
 __device__ __forceinline__ void store_out(OutT* dst, float x);
 template <>
@@ -141,6 +149,7 @@ swa_decode_kernel(const DecodeParams p) {
   const int G = p.n_q_heads / p.n_kv_heads;
   const int W = p.window;
 
+  wait_prior_grid();
   const long long pos = p.pos[b];
   if (pos < 0) {
     if (threadIdx.x == 0) raise_status(p.status, SWA_ERR_DEVICE_ARG);
@@ -386,6 +395,7 @@ swa_decode_kernel(const DecodeParams p) {
 template <int D, typename OutT>
 __global__ void __launch_bounds__(D < 32 ? 32 : D)
 swa_decode_combine_kernel(const DecodeParams p) {
+  wait_prior_grid();
   const size_t bh = blockIdx.x;
   const int dd = threadIdx.x;
   if (dd >= D) return;
@@ -416,28 +426,34 @@ cudaError_t launch_decode_t(const DecodeParams& p, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  dim3 grid(p.n_splits, p.n_kv_heads, p.batch);
-  if (p.cluster) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(NW * 32);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)p.n_splits;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, p);
+  if (p.cluster && p.n_splits > 8) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
   }
-  kern<<<grid, NW * 32, smem, stream>>>(p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || p.n_splits == 1) return e;
-  swa_decode_combine_kernel<D, OutT><<<(unsigned)((size_t)p.batch * p.n_q_heads), D < 32 ? 32 : D, 0,
-                                       stream>>>(p);
-  return cudaGetLastError();
+  dim3 grid(p.n_splits, p.n_kv_heads, p.batch);
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)p.n_splits;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(NW * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.cluster ? 2 : 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+  if (e != cudaSuccess || p.n_splits == 1 || p.cluster) return e;
+  cudaLaunchConfig_t ccfg = {};
+  ccfg.gridDim = dim3((unsigned)((size_t)p.batch * p.n_q_heads));
+  ccfg.blockDim = dim3(D < 32 ? 32 : D);
+  ccfg.stream = stream;
+  ccfg.attrs = attr;
+  ccfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&ccfg, swa_decode_combine_kernel<D, OutT>, p);
 }
 
 template <int D, typename OutT>
