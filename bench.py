@@ -48,11 +48,11 @@ METRIC = ("prefill tokens/s & TFLOP/s (% bf16 peak); decode tokens/s & HBM GB/s 
 # while the kernel source is the one that was profiled (sha256 prefix of the .cu file);
 # the summaries with the commands are under profiles/.
 PROFILED_TRAFFIC = {
-    "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "4a934635ab7980c7",
-                           "bytes": 67_203_840 + 5_355_264,
+    "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "924dc2b02db820b0",
+                           "bytes": 67_197_184 + 5_038_080,
                            "launch": "chunk 1 of 4 (every row sees 4096 keys)"},
-    "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "755fd51e78c93611",
-                          "bytes": 1_074_287_000 + 4_925_696, "launch": "one decode step"},
+    "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "7d6ddd2772e3e77d",
+                          "bytes": 1_074_321_000 + 4_719_872, "launch": "one decode step"},
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20

@@ -353,3 +353,20 @@ def test_planted_cache_mistakes_fail_the_invariant():
     np.testing.assert_allclose(chunked(False, False), ref, rtol=RTOL, atol=1e-12)
     assert np.abs(chunked(True, False) - ref).max() > 1e-3
     assert np.abs(chunked(False, True) - ref).max() > 1e-3
+
+
+def test_one_token_chunk_is_a_decode_step():
+    # a chunk of one token attends to the cache before its append plus itself:
+    # the same keys as a decode step, which appends first (section 2)
+    g = np.random.default_rng(9)
+    W, Hkv, Hq, d, pos = 8, 2, 4, 16, 13
+    q = g.standard_normal((1, 1, Hq, d))
+    k = g.standard_normal((1, 1, Hkv, d))
+    v = g.standard_normal((1, 1, Hkv, d))
+    a = oracle.RollingCache(1, Hkv, W, d)
+    for p in range(pos - W + 1, pos):
+        a.write(0, p, g.standard_normal((Hkv, d)), g.standard_normal((Hkv, d)))
+    b = a.copy()
+    pre = oracle.prefill_chunk(a, q, k, v, [pos], [1], 0.25)[0, 0]
+    dec = oracle.decode(b, q[:, 0], k[:, 0], v[:, 0], [pos], 0.25)[0]
+    np.testing.assert_allclose(pre, dec, rtol=0, atol=1e-14)
