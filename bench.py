@@ -48,7 +48,7 @@ METRIC = ("prefill tokens/s & TFLOP/s (% bf16 peak); decode tokens/s & HBM GB/s 
 # while the kernel source is the one that was profiled (sha256 prefix of the .cu file);
 # the summaries with the commands are under profiles/.
 PROFILED_TRAFFIC = {
-    "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "924dc2b02db820b0",
+    "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "0cdc3b2e8f72bfe1",
                            "bytes": 67_197_184 + 5_038_080,
                            "launch": "chunk 1 of 4 (every row sees 4096 keys)"},
     "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "7d6ddd2772e3e77d",

@@ -146,13 +146,14 @@ int encode_map(EncodeTiledFn fn, CUtensorMap* map, const void* ptr, int rank, co
   return SWA_OK;
 }
 
-// Progress words of trace builds (-DSWA_TRACE): host-mapped memory set by
+// Progress words of trace builds (-DSWA_TRACE, host-mapped memory) or the tile
+// counters of checked builds (-DSWA_TILE_COUNTERS, device memory), set by
 // swa_debug_set_trace; always NULL in normal builds.
 int* g_trace = nullptr;
 
 }  // namespace
 
-#ifdef SWA_TRACE
+#if defined(SWA_TRACE) || defined(SWA_TILE_COUNTERS)
 extern "C" SWA_API void swa_debug_set_trace(void* host_mapped) { g_trace = static_cast<int*>(host_mapped); }
 #endif
 

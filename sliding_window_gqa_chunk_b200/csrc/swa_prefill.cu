@@ -303,6 +303,9 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
         if (!ok) break;
         const uint32_t kdst = sK + sk * C::kTileBytes;
         tc::mbar_arrive_expect_tx(bar_k_full + 8 * sk, C::kTileBytes);
+#ifdef SWA_TILE_COUNTERS
+        if (p.trace != nullptr) atomicAdd(p.trace, 1);  // checked build: key tiles loaded
+#endif
         for (int cb = 0; cb < C::kColBlocks; ++cb) {
           if (is_cache)
             tc::tma_load_3d(kdst + cb * C::kBlockBytes, &maps.kc, cb * C::kBoxD, kbase,
@@ -492,6 +495,12 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
             if (kbase + k > t) sv[k] = -CUDART_INF_F;
         }
       }
+#ifdef SWA_TILE_COUNTERS
+      {  // checked build: (warp, tile) pairs with / without a masked key
+        const bool wm = __any_sync(0xffffffffu, masked);
+        if (lane == 0 && p.trace != nullptr) atomicAdd(p.trace + (wm ? 1 : 2), 1);
+      }
+#endif
 
       // P = exp2(scale * log2(e) * s - base) for the whole tile, written over
       // the first 64 columns of S_i; returns this thread's sum of the fp32 p.
