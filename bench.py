@@ -52,7 +52,7 @@ PROFILED_TRAFFIC = {
                            "bytes": 67_197_184 + 5_038_080,
                            "launch": "chunk 1 of 4 (every row sees 4096 keys)"},
     "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "7d6ddd2772e3e77d",
-                          "bytes": 1_074_321_000 + 4_719_872, "launch": "one decode step"},
+                          "bytes": 1_074_303_000 + 3_859_712, "launch": "one decode step"},
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
@@ -325,14 +325,18 @@ def run_prefill_e2e(run: PrefillRun, steps: int, warmup: int, flush):
     return sum(times) / len(times), h2d, d2h
 
 
-def decode_launches_per_call(dims, swa_mod):
-    """Kernels one swa_decode call launches.  Few (sequence, kv head) pairs
-    (batch x n_kv_heads < 64) run as one launch whose splits merge inside a
-    thread-block cluster; otherwise a split sweep is followed by a combine
-    kernel whenever the workspace holds per-split partials."""
-    if dims.batch * dims.n_kv_heads < 64:
+def decode_launches_per_call(dims, swa_mod=None):
+    """Kernels one swa_decode call launches (the library's split rule restated).
+    Few (sequence, kv head) pairs (batch x n_kv_heads < 64) run as one launch
+    whose splits merge inside a thread-block cluster.  Otherwise the W slots
+    are split into floor(592 / pairs) parts (at least 1, at most W / 64: one
+    wave of four 4-warp CTAs per SM on 148 SMs), and more than one split adds
+    a combine kernel."""
+    units = dims.batch * dims.n_kv_heads
+    if units < 64:
         return 1
-    return 1 if swa_mod.decode_workspace_size(dims) <= 16 else 2
+    splits = max(1, min(592 // units, -(-dims.window // 64)))
+    return 1 if splits == 1 else 2
 
 
 class DecodeRun:
@@ -576,7 +580,8 @@ def bench_ours(args, world, rank, local):
             "workload": DECODE_B64.name, "batch": DECODE_B64.batch,
             "tokens_per_s": round(world * DECODE_B64.batch / (dms_max / 1e3), 1),
             "ms_per_step": round(dms_max, 4),
-            "roofline": {"kernel": "swa_decode_kernel (+ combine)", "bound": "hbm",
+            "roofline": {"kernel": "swa_decode_kernel" + (" (+ combine)" if dec.launches_per_step > 1 else ""),
+                         "bound": "hbm",
                          "achieved": round(dec_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(dec_gbs / peaks["hbm_gbs"], 4),
                          "peak_source": f"{peaks['source']} hbm_gbs",

@@ -164,6 +164,12 @@ namespace swa {
 #ifndef SWA_DECODE_MAX_CLUSTER
 #define SWA_DECODE_MAX_CLUSTER 8
 #endif
+// Non-zero: the number of splits rounds down (at least this many), so that the
+// CTAs fit in one wave of resident 4-warp CTAs (a second, nearly empty wave
+// cost up to a third of the sweep); 0: rounds up.
+#ifndef SWA_DECODE_SPLIT_FLOOR
+#define SWA_DECODE_SPLIT_FLOOR 1
+#endif
 // 0: never merge splits in a cluster (always the workspace and the combine kernel)
 #ifndef SWA_DECODE_CLUSTER
 #define SWA_DECODE_CLUSTER 1
@@ -173,7 +179,8 @@ DecodeSplit decode_split(int batch, int n_q_heads, int n_kv_heads, int window) {
   const long long units = (long long)batch * n_kv_heads;
   // Workspace split: about four resident 128-thread CTAs per SM on a 148-SM
   // B200, each split a multiple of 64 slots (16 per warp); the per-split fp32
-  // partials are merged by a second kernel.
+  // partials are merged by a second kernel.  The workspace is sized for this
+  // count; the launch may use fewer splits (below).
   const long long target = 148LL * 4;
   long long splits = (target + units - 1) / units;
   const long long max_splits = (window + 63) / 64;
@@ -187,6 +194,18 @@ DecodeSplit decode_split(int batch, int n_q_heads, int n_kv_heads, int window) {
   s.ws_splits = s.n_splits;
   s.warps = 4;
   s.cluster = 0;
+#if SWA_DECODE_SPLIT_FLOOR
+  {
+    long long fs = target / units;
+    if (fs > max_splits) fs = max_splits;
+    if (fs < SWA_DECODE_SPLIT_FLOOR) fs = SWA_DECODE_SPLIT_FLOOR;
+    if (fs > splits) fs = splits;
+    long long fper = (window + fs - 1) / fs;
+    fper = (fper + 63) / 64 * 64;
+    s.slots_per_split = (int)fper;
+    s.n_splits = (int)((window + fper - 1) / fper);
+  }
+#endif
   if (SWA_DECODE_CLUSTER && units < 64) {
     // Few (sequence, kv head) pairs: the sweep is latency-bound, so each pair
     // gets one cluster of up to 8 CTAs of 16 warps (8 for groups above 8
