@@ -104,7 +104,10 @@ SWA_API int swa_cache_append(const swa_dims* dims, void* k_cache, void* v_cache,
  *   out               [B][max_tokens][Hq][d], bf16 or f32 per dims->out_dtype;
  *                     rows t >= n_tokens[b] are not written
  *   q                 [B][max_tokens][Hq][d] bf16
- *   k, v              [B][max_tokens][Hkv][d] bf16 (the chunk's own keys/values)
+ *   k, v              [B][max_tokens][Hkv][d] bf16 (the chunk's own keys/values);
+ *                     rows [n_tokens[b], max_tokens) must hold finite values
+ *                     (they are loaded with their tile and masked, and a NaN
+ *                     there would reach the output through 0 * NaN)
  *   max_tokens        1 <= max_tokens <= W
  *   k_cache, v_cache  [B][Hkv][W][d] bf16, read only; slots must hold the
  *                     positions earlier appends put there.  A sequence whose
@@ -119,9 +122,11 @@ SWA_API int swa_prefill_chunk(const swa_dims* dims, void* out, const void* q, co
                       const int32_t* n_tokens, void* stream);
 
 /*
- * swa_decode_workspace_size - bytes of device scratch swa_decode needs for
- * these dims (fp32 partial results of the split cache sweep).  Depends only on
- * dims.  Returns 0 for invalid dims.
+ * swa_decode_workspace_size - bytes of device scratch swa_decode may use for
+ * these dims (fp32 partial results of a split cache sweep).  Depends only on
+ * dims.  Some dims use none of it (one split per sequence and kv head, or
+ * splits merged inside a thread-block cluster); the size is still reported so
+ * that it stays a function of the dims.  Returns 0 for invalid dims.
  */
 SWA_API size_t swa_decode_workspace_size(const swa_dims* dims);
 
