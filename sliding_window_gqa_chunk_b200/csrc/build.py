@@ -51,6 +51,7 @@ def build(force: bool = False, verbose: bool = False, defines=(), out: str | Non
     target = out or LIB
     if not force and out is None and up_to_date():
         return LIB
+    os.makedirs(os.path.dirname(os.path.abspath(target)), exist_ok=True)
     tmp = target + f".tmp{os.getpid()}"
     cmd = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",
