@@ -325,18 +325,10 @@ def run_prefill_e2e(run: PrefillRun, steps: int, warmup: int, flush):
     return sum(times) / len(times), h2d, d2h
 
 
-def decode_launches_per_call(dims, swa_mod=None):
-    """Kernels one swa_decode call launches (the library's split rule restated).
-    Few (sequence, kv head) pairs (batch x n_kv_heads < 64) run as one launch
-    whose splits merge inside a thread-block cluster.  Otherwise the W slots
-    are split into floor(592 / pairs) parts (at least 1, at most W / 64: one
-    wave of four 4-warp CTAs per SM on 148 SMs), and more than one split adds
-    a combine kernel."""
-    units = dims.batch * dims.n_kv_heads
-    if units < 64:
-        return 1
-    splits = max(1, min(592 // units, -(-dims.window // 64)))
-    return 1 if splits == 1 else 2
+def decode_launches_per_call(dims, swa_mod):
+    """Kernels one swa_decode call launches for these dims, as the library
+    reports them (swa_decode_launch_info)."""
+    return swa_mod.decode_launch_info(dims)[1]
 
 
 class DecodeRun:

@@ -131,6 +131,18 @@ SWA_API int swa_prefill_chunk(const swa_dims* dims, void* out, const void* q, co
 SWA_API size_t swa_decode_workspace_size(const swa_dims* dims);
 
 /*
+ * swa_decode_launch_info - how swa_decode runs for these dims, for callers
+ * that count kernels (CUDA graphs, profilers).  Host only; enqueues nothing.
+ *   n_splits    receives the number of parts the W slots of one (sequence,
+ *               kv head) are split into (one CTA each)
+ *   n_launches  receives the number of kernels one swa_decode call launches:
+ *               1, or 2 when a combine kernel merges per-split partials
+ * Either pointer may be NULL.  Returns SWA_OK, or the same codes as
+ * swa_decode for invalid dims.
+ */
+SWA_API int swa_decode_launch_info(const swa_dims* dims, int32_t* n_splits, int32_t* n_launches);
+
+/*
  * swa_decode - one generated token per sequence (token-by-token generation,
  * Rolling Buffer Cache paragraph).  The new key/value of position pos[b] is
  * written to slot pos[b] mod W, then the query attends over the cache: the

@@ -115,6 +115,8 @@ def load_library() -> ctypes.CDLL:
         lib.swa_prefill_chunk.restype = ctypes.c_int
         lib.swa_decode_workspace_size.argtypes = [D]
         lib.swa_decode_workspace_size.restype = ctypes.c_size_t
+        lib.swa_decode_launch_info.argtypes = [D, ctypes.POINTER(I32), ctypes.POINTER(I32)]
+        lib.swa_decode_launch_info.restype = ctypes.c_int
         lib.swa_decode.argtypes = [D, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         lib.swa_decode.restype = ctypes.c_int
         lib.swa_decode_static.argtypes = [D, P, P, P, P, P, P, P, P]
@@ -182,6 +184,14 @@ def prefill_chunk(dims: Dims, out, q, k, v, k_cache, v_cache, start_pos, n_token
 def decode_workspace_size(dims: Dims) -> int:
     cd = dims.c()
     return int(load_library().swa_decode_workspace_size(ctypes.byref(cd)))
+
+
+def decode_launch_info(dims: Dims):
+    """(n_splits, n_launches) of swa_decode for these dims (host only)."""
+    cd = dims.c()
+    ns, nl = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(load_library().swa_decode_launch_info(ctypes.byref(cd), ctypes.byref(ns), ctypes.byref(nl)))
+    return int(ns.value), int(nl.value)
 
 
 def decode(dims: Dims, out, q, k_new, v_new, k_cache, v_cache, pos, workspace,

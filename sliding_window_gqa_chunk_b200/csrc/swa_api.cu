@@ -333,6 +333,17 @@ size_t swa_decode_workspace_size(const swa_dims* dims) {
   return bh * dims->head_dim * sizeof(float) + bh * 2 * sizeof(float);
 }
 
+int swa_decode_launch_info(const swa_dims* dims, int32_t* n_splits, int32_t* n_launches) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  const swa::DecodeSplit sp =
+      swa::decode_split(dims->batch, dims->n_q_heads, dims->n_kv_heads, dims->window);
+  if (n_splits) *n_splits = sp.n_splits;
+  // a cluster merges its splits in-kernel; otherwise several splits need the combine kernel
+  if (n_launches) *n_launches = (sp.n_splits > 1 && !sp.cluster) ? 2 : 1;
+  return ok();
+}
+
 int swa_decode(const swa_dims* dims, void* out, const void* q, const void* k_new, const void* v_new,
                void* k_cache, void* v_cache, const int32_t* pos, void* workspace, size_t workspace_bytes,
                void* stream) {

@@ -134,3 +134,23 @@ def test_python_binding_refuses_to_run_without_the_library(tmp_path, monkeypatch
     monkeypatch.setattr(swa, "_LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         swa.load_library()
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,W,expect", [
+    (1, 32, 8, 4096, (8, 1)),     # 8 pairs: one cluster of 8 CTAs per pair, merged in-kernel
+    (4, 32, 8, 4096, (8, 1)),     # 32 pairs: still clustered
+    (16, 32, 8, 4096, (4, 2)),    # 128 pairs: floor(592 / 128) = 4 splits + combine
+    (64, 32, 8, 4096, (1, 1)),    # 512 pairs: one split, no combine
+    (128, 32, 8, 4096, (1, 1)),
+    (2, 8, 2, 300, (2, 1)),       # cluster of 2 CTAs (300 slots, 256 per 16-warp CTA sweep)
+    (3, 12, 4, 100, (1, 1)),      # one CTA covers the window
+])
+def test_decode_launch_info_follows_the_split_rule(B, Hq, Hkv, W, expect):
+    d = swa.Dims(B, Hq, Hkv, 128, W, 0.1, "bf16")
+    assert swa.decode_launch_info(d) == expect
+
+
+def test_decode_launch_info_rejects_bad_dims(lib):
+    d = dims(batch=1, n_kv_heads=3, n_q_heads=8, window=64)   # Hq % Hkv != 0
+    rc = lib.swa_decode_launch_info(ctypes.byref(d), None, None)
+    assert rc == swa.SWA_ERR_UNSUPPORTED
