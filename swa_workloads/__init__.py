@@ -28,7 +28,7 @@ from __future__ import annotations
 
 import dataclasses
 import math
-from typing import Iterator, List, Optional, Sequence, Tuple
+from typing import Optional, Sequence, Tuple
 
 import torch
 
@@ -153,35 +153,6 @@ def prefill_inputs(wl: PrefillWorkload, device: str = "cpu"):
     return q, k, v
 
 
-def chunk_schedule(lengths: Sequence[int], chunk: int) -> List[Tuple[List[int], List[int]]]:
-    """Calls of a batched chunked prefill, in issue order.
-
-    Call c covers tokens [c*chunk, (c+1)*chunk) of every sequence that still has
-    tokens there.  Returns a list of (start_pos[B], n_tokens[B]); a sequence
-    with nothing left in call c has n_tokens 0.
-    """
-    n_calls = max((n + chunk - 1) // chunk for n in lengths)
-    out = []
-    for c in range(n_calls):
-        starts, counts = [], []
-        for n in lengths:
-            st = c * chunk
-            starts.append(st)
-            counts.append(max(0, min(chunk, n - st)))
-        out.append((starts, counts))
-    return out
-
-
-def slice_chunk(x: torch.Tensor, start: int, count: int) -> torch.Tensor:
-    """Rows [start, start+count) of [B, L, H, d], zero-padded to ``count`` rows."""
-    B, L = x.shape[0], x.shape[1]
-    out = torch.zeros((B, count) + tuple(x.shape[2:]), dtype=x.dtype, device=x.device)
-    hi = min(L, start + count)
-    if hi > start:
-        out[:, : hi - start] = x[:, start:hi]
-    return out
-
-
 def tiny_inputs(seed: int = TINY_PREFILL.seed):
     """Config 1 draws: q,k,v for each of the 3 chunks, then q,k,v for each of 4 steps.
 
@@ -254,6 +225,3 @@ def random_case(seed: int, B: int, L: int, Hq: int, Hkv: int, d: int,
     return q, k, v
 
 
-def iter_decode_steps(wl: DecodeWorkload, steps: int, device: str = "cpu") -> Iterator:
-    for i in range(steps):
-        yield decode_step_inputs(wl, i, 0, device)
