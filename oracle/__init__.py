@@ -24,9 +24,9 @@ It follows Mistral 7B, section 2 "Architectural details":
 * Token-by-token generation: ``decode`` writes the new key/value at slot
   pos mod W and attends over the cache afterwards.
 
-Readings where the pages are silent or ambiguous (window bounds, GQA grouping,
-cache-before-append for chunks, append-before-attend for decode) are the ones
-stated above; each is listed in the design doc.
+Where the pages are silent or ambiguous (window bounds, GQA grouping,
+cache-before-append for chunks, append-before-attend for decode), this module
+follows the readings stated above.
 """
 from __future__ import annotations
 
