@@ -5,8 +5,8 @@ oracle: it rebuilds the visible set of every query from scratch by walking the
 whole token history, and evaluates the softmax with ``math.exp`` on Python
 floats, one (row, head) at a time.  Meant for a few dozen tokens at most.
 
-Mistral 7B, section 2: token i sees tokens j in (i - W, i] (Figure 1 caption:
-"at most W tokens"); query head h reads kv head h // (Hq // Hkv).
+Mistral 7B, section 2: token i sees tokens j in (i - W, i], at most W of them
+(Figure 1 caption); query head h reads kv head h // (Hq // Hkv).
 """
 from __future__ import annotations
 
