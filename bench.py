@@ -238,6 +238,7 @@ class PrefillRun:
         self.out = torch.empty((1, self.L, s.n_q_heads, s.head_dim), dtype=self.dims.torch_out_dtype,
                                device=device)
         self.kc, self.vc = swa.new_cache(self.dims, device)
+        self.ws = swa.prefill_workspace(self.dims, self.chunk, device)
         n_calls = (self.L + self.chunk - 1) // self.chunk
         self.starts = [torch.tensor([c * self.chunk], dtype=torch.int32, device=device)
                        for c in range(n_calls)]
@@ -259,7 +260,8 @@ class PrefillRun:
         q, k, v, o = self.views[c]
         if events is not None:
             events[c][0].record()
-        self.swa.prefill_chunk(self.dims, o, q, k, v, self.kc, self.vc, self.starts[c], self.counts[c])
+        self.swa.prefill_chunk(self.dims, o, q, k, v, self.kc, self.vc, self.starts[c], self.counts[c],
+                               workspace=self.ws)
         if events is not None:
             events[c][1].record()
         self.swa.cache_append(self.dims, self.kc, self.vc, k, v, self.starts[c], self.counts[c])
@@ -347,7 +349,7 @@ class DecodeRun:
         self.inputs = [decode_step_inputs(wl, i, 0, device=device) for i in range(4)]
         self.out = torch.empty((wl.batch, s.n_q_heads, s.head_dim), dtype=self.dims.torch_out_dtype,
                                device=device)
-        self.ws = torch.empty(swa.decode_workspace_size(self.dims), dtype=torch.uint8, device=device)
+        self.ws = swa.decode_workspace(self.dims, device)
         self.i = 0
         B, W, Hkv, d, Hq = wl.batch, s.window, s.n_kv_heads, s.head_dim, s.n_q_heads
         out_b = 4 if out_dtype == "f32" else 2
@@ -383,6 +385,7 @@ class VarlenRun:
         self.dims = swa.Dims(B, s.n_q_heads, s.n_kv_heads, s.head_dim, s.window, wl.scale, out_dtype)
         q, k, v = prefill_inputs(wl, device=device)
         self.kc, self.vc = swa.new_cache(self.dims, device)
+        self.ws = swa.prefill_workspace(self.dims, C, device)
         self.n_calls = (max(wl.lengths) + C - 1) // C
         self.calls = []
         flops = 0.0
@@ -411,7 +414,8 @@ class VarlenRun:
         for c, (qc, kc, vc, out, sp, nt) in enumerate(self.calls):
             if events is not None:
                 events[c][0].record()
-            self.swa.prefill_chunk(self.dims, out, qc, kc, vc, self.kc, self.vc, sp, nt)
+            self.swa.prefill_chunk(self.dims, out, qc, kc, vc, self.kc, self.vc, sp, nt,
+                                   workspace=self.ws)
             if events is not None:
                 events[c][1].record()
             self.swa.cache_append(self.dims, self.kc, self.vc, kc, vc, sp, nt)
@@ -441,7 +445,7 @@ class Decode32Run:
         self.v = torch.randn((B, s.n_kv_heads, s.head_dim), generator=g, device=device, dtype=torch.bfloat16)
         self.out = torch.empty((B, s.n_q_heads, s.head_dim), dtype=self.dims.torch_out_dtype, device=device)
         self.pos = decode_positions(wl, device=device)
-        self.ws = torch.empty(max(16, swa.decode_workspace_size(self.dims)), dtype=torch.uint8, device=device)
+        self.ws = swa.decode_workspace(self.dims, device)
         out_b = 4 if out_dtype == "f32" else 2
         per_layer = B * (2 * s.window * s.n_kv_heads * s.head_dim * 2 + s.n_q_heads * s.head_dim * 2 +
                          2 * s.n_kv_heads * s.head_dim * 2 * 2 + s.n_q_heads * s.head_dim * out_b)
@@ -597,13 +601,15 @@ def bench_ours(args, world, rank, local):
         # dense causal comparator on the same inputs: one chunk of 16384, W = 16384
         dense_dims = swa.Dims(1, 32, 8, 128, 16384, wl.scale, "bf16")
         dkc, dvc = swa.new_cache(dense_dims, dev)
+        dws = swa.prefill_workspace(dense_dims, 16384, dev)
         zero = torch.zeros(1, dtype=torch.int32, device=dev)
         full = torch.tensor([16384], dtype=torch.int32, device=dev)
 
         def dense_step(ev):
             if ev is not None:
                 ev[0][0].record()
-            swa.prefill_chunk(dense_dims, run.out, run.q, run.k, run.v, dkc, dvc, zero, full)
+            swa.prefill_chunk(dense_dims, run.out, run.q, run.k, run.v, dkc, dvc, zero, full,
+                              workspace=dws)
             if ev is not None:
                 ev[0][1].record()
 
@@ -673,35 +679,45 @@ def bench_ours(args, world, rank, local):
 # CPU oracle (reference arm and cpu_baseline)
 # ----------------------------------------------------------------------------
 
-def oracle_sample(wl, rows: int, q, k, v):
-    """The oracle on `rows` query tokens of the last chunk (all heads), each
-    attending to its full window: returns seconds."""
+def oracle_rows(wl, seed: int = 0):
+    """Query rows of the whole prompt in a seeded random order: timing the
+    oracle on a prefix of this list samples every chunk in proportion to its
+    rows, each row with its own min(i + 1, W) keys, so rows / second estimates
+    the whole prompt's rate."""
+    g = torch.Generator().manual_seed(seed)
+    return torch.randperm(wl.lengths[0], generator=g).tolist()
+
+
+def oracle_sample(wl, rows, q, k, v):
+    """The oracle on the given query rows (all heads, each row against its
+    window of keys from the full history): returns seconds."""
     import numpy as np
     import oracle
-    L, W = wl.lengths[0], wl.shape.window
-    st = L - wl.chunk                      # last chunk: every row sees W keys
-    lo = st - W + 1
-    qs = q[0, st:st + rows]
-    ks = k[0, max(0, lo):st + rows]
-    vs = v[0, max(0, lo):st + rows]
+    W = wl.shape.window
     t0 = time.perf_counter()
-    oracle.attend(qs, np.arange(st, st + rows), ks, vs, np.arange(max(0, lo), st + rows), W,
-                  wl.scale)
+    for i in rows:
+        lo = max(0, i - W + 1)
+        oracle.attend(q[0, i:i + 1], [i], k[0, lo:i + 1], v[0, lo:i + 1], np.arange(lo, i + 1), W,
+                      wl.scale)
     return time.perf_counter() - t0
+
+
+def sample_note(n_rows, wl):
+    return (f"{n_rows} query tokens drawn uniformly at random from the {wl.lengths[0]}-token prompt "
+            f"(all 32 heads, each row against its own min(i+1, {wl.shape.window}) keys), float64 C "
+            f"oracle, OpenMP over heads")
 
 
 def cpu_baseline(wl, budget_s=12.0):
     import oracle
     q, k, v = prefill_inputs(wl, device="cpu")
-    rows, spent, total_rows = 64, 0.0, 0
-    while spent < budget_s and total_rows + rows <= wl.chunk:
-        spent += oracle_sample(wl, rows, q, k, v)
-        total_rows += rows
-        rows = min(rows * 2, 512)
-    return {"value": round(total_rows / spent, 2), "unit": "tokens/s", "cores": oracle.max_threads(),
-            "kind": "oracle",
-            "sample": f"{total_rows} query tokens of the last 4096-token chunk (all 32 heads, "
-                      f"4096 keys each), float64 C oracle, OpenMP"}
+    order = oracle_rows(wl)
+    done, spent, batch = 0, 0.0, 32
+    while spent < budget_s and done + batch <= len(order):
+        spent += oracle_sample(wl, order[done:done + batch], q, k, v)
+        done += batch
+    return {"value": round(done / spent, 2), "unit": "tokens/s", "cores": oracle.max_threads(),
+            "kind": "oracle", "sample": sample_note(done, wl)}
 
 
 def bench_reference(args, world, rank):
@@ -712,13 +728,16 @@ def bench_reference(args, world, rank):
     wl = PREFILL_16K
     q, k, v = prefill_inputs(wl, device="cpu")
     rows = args.ref_rows
-    for _ in range(args.warmup):
-        oracle_sample(wl, rows, q, k, v)
-    times = [oracle_sample(wl, rows, q, k, v) for _ in range(args.steps)]
+    order = oracle_rows(wl, seed=1)
+    for i in range(args.warmup):
+        oracle_sample(wl, order[i * rows:(i + 1) * rows], q, k, v)
+    times = []
+    for i in range(args.steps):
+        a = ((args.warmup + i) * rows) % len(order)
+        times.append(oracle_sample(wl, order[a:a + rows], q, k, v))
     per = sum(times) / len(times)
     value = rows / per
-    sample = (f"{rows} query tokens of the last 4096-token chunk per step (all 32 heads, 4096 "
-              f"keys each), float64 C oracle, OpenMP")
+    sample = sample_note(rows, wl) + " per step"
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

@@ -94,6 +94,14 @@ SWA_API int swa_cache_append(const swa_dims* dims, void* k_cache, void* v_cache,
                      const int32_t* start_pos, const int32_t* n_tokens, void* stream);
 
 /*
+ * swa_prefill_workspace_size - bytes of device scratch swa_prefill_chunk may
+ * use for these dims and this max_tokens: per-row partial results of query
+ * tiles whose key range is split across CTAs, and the work and merge counters.
+ * Depends only on its arguments.  Returns 0 for invalid arguments.
+ */
+SWA_API size_t swa_prefill_workspace_size(const swa_dims* dims, int32_t max_tokens);
+
+/*
  * swa_prefill_chunk - attention of one prefill chunk (Pre-fill and Chunking
  * paragraph, Figure 3).  Query row t of sequence b sits at position
  * i = start_pos[b] + t and attends to
@@ -113,13 +121,25 @@ SWA_API int swa_cache_append(const swa_dims* dims, void* k_cache, void* v_cache,
  *                     positions earlier appends put there.  A sequence whose
  *                     start_pos is 0 reads nothing from them.
  *   start_pos, n_tokens  device int32[B], as in swa_cache_append
+ *   workspace         NULL (with workspace_bytes 0), or device scratch of at
+ *                     least swa_prefill_workspace_size(dims, max_tokens) bytes,
+ *                     16-byte aligned, ZERO-FILLED before its first use (every
+ *                     call leaves it zero-filled again, so this is needed once).
+ *                     With a workspace the kernel runs one CTA per SM that
+ *                     takes query tiles from a shared counter and splits the
+ *                     key ranges of the last tiles across CTAs (their partial
+ *                     softmax results are merged by log-sum-exp); without one
+ *                     it launches one CTA per query tile and head pair.  The
+ *                     results agree within rounding.  Calls that may overlap
+ *                     on the GPU need separate workspaces.
  * The softmax is computed in fp32 from bf16 q.k products accumulated in fp32;
  * the probabilities are rounded to bf16 for the P.V product.
  */
 SWA_API int swa_prefill_chunk(const swa_dims* dims, void* out, const void* q, const void* k,
                       const void* v, int32_t max_tokens, const void* k_cache,
                       const void* v_cache, const int32_t* start_pos,
-                      const int32_t* n_tokens, void* stream);
+                      const int32_t* n_tokens, void* workspace, size_t workspace_bytes,
+                      void* stream);
 
 /*
  * swa_decode_workspace_size - bytes of device scratch swa_decode may use for
@@ -173,9 +193,11 @@ SWA_API int swa_decode(const swa_dims* dims, void* out, const void* q, const voi
  * and ownership) but no workspace.
  *   - The decode scratch comes from one array built into the library,
  *     4 MiB (4194304 bytes) per device, held by every GPU that loads the
- *     library until the process exits.  Dims whose swa_decode_workspace_size
- *     exceeds 4 MiB are rejected with SWA_ERR_WORKSPACE_TOO_SMALL and nothing
- *     is enqueued.
+ *     library until the process exits.  A launch whose splits merge through
+ *     memory needs B * Hq * n_splits * (d + 2) * 4 bytes of it (n_splits from
+ *     swa_decode_launch_info; none when that reports one launch).  Dims that
+ *     need more than 4 MiB are rejected with SWA_ERR_WORKSPACE_TOO_SMALL and
+ *     nothing is enqueued.
  *   - The call allocates nothing.  Its first call on each device looks up the
  *     array's device address, with that device current; make that first call
  *     before any stream capture begins.

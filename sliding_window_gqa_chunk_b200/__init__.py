@@ -17,10 +17,11 @@ Typical use for one layer::
     dims = Dims(batch=B, n_q_heads=32, n_kv_heads=8, head_dim=128, window=4096,
                 scale=128 ** -0.5)
     kc, vc = new_cache(dims)                       # zeroed [B, Hkv, W, d] bf16
+    pws = prefill_workspace(dims, max_tokens=4096)  # zeroed, reused by every call
     for chunk ...:                                  # prompt, chunk by chunk
-        prefill_chunk(dims, out, q, k, v, kc, vc, start_pos, n_tokens)
+        prefill_chunk(dims, out, q, k, v, kc, vc, start_pos, n_tokens, workspace=pws)
         cache_append(dims, kc, vc, k, v, start_pos, n_tokens)
-    ws = torch.empty(decode_workspace_size(dims), dtype=torch.uint8, device="cuda")
+    ws = decode_workspace(dims)
     decode(dims, out1, q1, k1, v1, kc, vc, pos, ws)  # one token per sequence
 """
 from __future__ import annotations
@@ -35,7 +36,8 @@ import torch
 
 __all__ = [
     "Dims", "SwaError", "load_library", "library_path", "cache_append", "prefill_chunk",
-    "decode", "decode_static", "decode_workspace_size", "device_status", "new_cache", "abi_version",
+    "decode", "decode_static", "decode_workspace_size", "decode_workspace", "decode_launch_info",
+    "prefill_workspace_size", "prefill_workspace", "device_status", "new_cache", "abi_version",
     "SWA_OK", "SWA_ERR_INVALID_ARG", "SWA_ERR_UNSUPPORTED", "SWA_ERR_WORKSPACE_TOO_SMALL",
     "SWA_ERR_CUDA", "SWA_ERR_TIMEOUT", "SWA_ERR_DEVICE_ARG",
 ]
@@ -111,7 +113,9 @@ def load_library() -> ctypes.CDLL:
         D = ctypes.POINTER(_CDims)
         lib.swa_cache_append.argtypes = [D, P, P, P, P, I32, P, P, P]
         lib.swa_cache_append.restype = ctypes.c_int
-        lib.swa_prefill_chunk.argtypes = [D, P, P, P, P, I32, P, P, P, P, P]
+        lib.swa_prefill_workspace_size.argtypes = [D, I32]
+        lib.swa_prefill_workspace_size.restype = ctypes.c_size_t
+        lib.swa_prefill_chunk.argtypes = [D, P, P, P, P, I32, P, P, P, P, P, ctypes.c_size_t, P]
         lib.swa_prefill_chunk.restype = ctypes.c_int
         lib.swa_decode_workspace_size.argtypes = [D]
         lib.swa_decode_workspace_size.restype = ctypes.c_size_t
@@ -172,18 +176,40 @@ def cache_append(dims: Dims, k_cache, v_cache, k, v, start_pos, n_tokens, stream
         _ptr(start_pos), _ptr(n_tokens), _stream(stream)))
 
 
-def prefill_chunk(dims: Dims, out, q, k, v, k_cache, v_cache, start_pos, n_tokens,
-                  stream=None) -> None:
-    """swa_prefill_chunk: out [B, T, Hq, d] = attention of chunk q over (cache + chunk k/v)."""
+def prefill_workspace_size(dims: Dims, max_tokens: int) -> int:
     cd = dims.c()
+    return int(load_library().swa_prefill_workspace_size(ctypes.byref(cd), int(max_tokens)))
+
+
+def prefill_workspace(dims: Dims, max_tokens: int, device="cuda") -> torch.Tensor:
+    """A zero-filled prefill workspace for these dims (reusable by every later
+    call with the same dims on the same stream; calls leave it zero-filled)."""
+    return torch.zeros(prefill_workspace_size(dims, max_tokens), dtype=torch.uint8, device=device)
+
+
+def prefill_chunk(dims: Dims, out, q, k, v, k_cache, v_cache, start_pos, n_tokens,
+                  workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """swa_prefill_chunk: out [B, T, Hq, d] = attention of chunk q over (cache + chunk k/v).
+
+    ``workspace`` (from ``prefill_workspace``) lets the kernel run persistently
+    and split the key ranges of its last query tiles across SMs; without it the
+    call launches one CTA per query tile and head pair."""
+    cd = dims.c()
+    ws_bytes = 0 if workspace is None else int(workspace.numel() * workspace.element_size())
     _check(load_library().swa_prefill_chunk(
         ctypes.byref(cd), _ptr(out), _ptr(q), _ptr(k), _ptr(v), int(q.shape[1]),
-        _ptr(k_cache), _ptr(v_cache), _ptr(start_pos), _ptr(n_tokens), _stream(stream)))
+        _ptr(k_cache), _ptr(v_cache), _ptr(start_pos), _ptr(n_tokens), _ptr(workspace),
+        ws_bytes, _stream(stream)))
 
 
 def decode_workspace_size(dims: Dims) -> int:
     cd = dims.c()
     return int(load_library().swa_decode_workspace_size(ctypes.byref(cd)))
+
+
+def decode_workspace(dims: Dims, device="cuda") -> torch.Tensor:
+    """A zero-filled decode workspace of decode_workspace_size(dims) bytes."""
+    return torch.zeros(decode_workspace_size(dims), dtype=torch.uint8, device=device)
 
 
 def decode_launch_info(dims: Dims):

@@ -146,6 +146,105 @@ int encode_map(EncodeTiledFn fn, CUtensorMap* map, const void* ptr, int rank, co
   return SWA_OK;
 }
 
+// The five TMA descriptors of a prefill call depend only on the tensors'
+// addresses and the shape, so they are kept for repeated calls (a prompt's
+// chunks, a decode loop that feeds one-token chunks): a small cache, replaced
+// round robin, keyed by device, pointers and shape.
+struct MapKey {
+  int device;
+  const void* ptr[5];
+  int batch, n_q_heads, n_kv_heads, head_dim, window, max_tokens;
+  bool operator==(const MapKey& o) const {
+    return device == o.device && memcmp(ptr, o.ptr, sizeof(ptr)) == 0 && batch == o.batch &&
+           n_q_heads == o.n_q_heads && n_kv_heads == o.n_kv_heads && head_dim == o.head_dim &&
+           window == o.window && max_tokens == o.max_tokens;
+  }
+};
+constexpr int kMapCacheSize = 16;
+std::mutex g_map_mu;
+MapKey g_map_keys[kMapCacheSize];
+swa::PrefillMaps g_map_vals[kMapCacheSize];
+int g_map_used = 0;
+int g_map_next = 0;
+
+#ifdef SWA_TEST_FAULTS
+// Checked build for the host-side fault test: when set, the next descriptor
+// encoding fails as if the driver had refused it (and the cache is bypassed).
+int g_fail_encode = 0;
+extern "C" SWA_API void swa_debug_fail_encode(int on) { g_fail_encode = on; }
+#endif
+
+int prefill_maps(int device, const swa_dims* dims, int max_tokens, const void* q, const void* k,
+                 const void* v, const void* k_cache, const void* v_cache, swa::PrefillMaps* out) {
+#ifdef SWA_TEST_FAULTS
+  if (g_fail_encode)
+    return fail(SWA_ERR_CUDA, "cuTensorMapEncodeTiled(q) failed with CUresult %d (injected)",
+                (int)CUDA_ERROR_INVALID_VALUE);
+#endif
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.device = device;
+  key.ptr[0] = q;
+  key.ptr[1] = k;
+  key.ptr[2] = v;
+  key.ptr[3] = k_cache;
+  key.ptr[4] = v_cache;
+  key.batch = dims->batch;
+  key.n_q_heads = dims->n_q_heads;
+  key.n_kv_heads = dims->n_kv_heads;
+  key.head_dim = dims->head_dim;
+  key.window = dims->window;
+  key.max_tokens = max_tokens;
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    for (int i = 0; i < g_map_used; ++i)
+      if (g_map_keys[i] == key) {
+        *out = g_map_vals[i];
+        return SWA_OK;
+      }
+  }
+  EncodeTiledFn enc = nullptr;
+  int rc = get_encode(&enc);
+  if (rc) return rc;
+  const int B = dims->batch, Hq = dims->n_q_heads, Hkv = dims->n_kv_heads, D = dims->head_dim;
+  const int W = dims->window;
+  int box_d = 0, swz = 0;
+  swa::prefill_map_geometry(D, &box_d, &swz);
+  swa::PrefillMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  const cuuint64_t es = 2;  // bf16
+  {
+    cuuint64_t dims4[4] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)max_tokens, (cuuint64_t)B};
+    cuuint64_t str4[3] = {D * es, (cuuint64_t)Hq * D * es, (cuuint64_t)max_tokens * Hq * D * es};
+    cuuint32_t box4[4] = {(cuuint32_t)box_d, 1, 128, 1};
+    if ((rc = encode_map(enc, &maps.q, q, 4, dims4, str4, box4, swz, "q"))) return rc;
+  }
+  {
+    cuuint64_t dims4[4] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)max_tokens, (cuuint64_t)B};
+    cuuint64_t str4[3] = {D * es, (cuuint64_t)Hkv * D * es, (cuuint64_t)max_tokens * Hkv * D * es};
+    cuuint32_t box4[4] = {(cuuint32_t)box_d, 1, 128, 1};
+    if ((rc = encode_map(enc, &maps.k, k, 4, dims4, str4, box4, swz, "k"))) return rc;
+    if ((rc = encode_map(enc, &maps.v, v, 4, dims4, str4, box4, swz, "v"))) return rc;
+  }
+  {
+    cuuint64_t dims3[3] = {(cuuint64_t)D, (cuuint64_t)W, (cuuint64_t)B * Hkv};
+    cuuint64_t str3[2] = {D * es, (cuuint64_t)W * D * es};
+    cuuint32_t box3[3] = {(cuuint32_t)box_d, 128, 1};
+    if ((rc = encode_map(enc, &maps.kc, k_cache, 3, dims3, str3, box3, swz, "k_cache"))) return rc;
+    if ((rc = encode_map(enc, &maps.vc, v_cache, 3, dims3, str3, box3, swz, "v_cache"))) return rc;
+  }
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    const int i = g_map_next;
+    g_map_keys[i] = key;
+    g_map_vals[i] = maps;
+    g_map_next = (g_map_next + 1) % kMapCacheSize;
+    if (g_map_used < kMapCacheSize) ++g_map_used;
+  }
+  *out = maps;
+  return SWA_OK;
+}
+
 // Progress words of trace builds (-DSWA_TRACE, host-mapped memory) or the tile
 // counters of checked builds (-DSWA_TILE_COUNTERS, device memory), set by
 // swa_debug_set_trace; always NULL in normal builds.
@@ -153,17 +252,14 @@ int* g_trace = nullptr;
 
 }  // namespace
 
-#if defined(SWA_TRACE) || defined(SWA_TILE_COUNTERS)
+#if defined(SWA_TRACE) || defined(SWA_TILE_COUNTERS) || defined(SWA_TEST_FAULTS)
 extern "C" SWA_API void swa_debug_set_trace(void* host_mapped) { g_trace = static_cast<int*>(host_mapped); }
 #endif
 
 namespace swa {
 
-// Largest thread-block cluster of the decode's split merge (8 is the portable
-// limit; 16 needs the non-portable opt-in, set at launch).
-#ifndef SWA_DECODE_MAX_CLUSTER
-#define SWA_DECODE_MAX_CLUSTER 8
-#endif
+// Largest thread-block cluster of the decode's split merge (the portable limit).
+constexpr int kDecodeMaxCluster = 8;
 // Non-zero: the number of splits rounds down (at least this many), so that the
 // CTAs fit in one wave of resident 4-warp CTAs (a second, nearly empty wave
 // cost up to a third of the sweep); 0: rounds up.
@@ -213,7 +309,7 @@ DecodeSplit decode_split(int batch, int n_q_heads, int n_kv_heads, int window) {
     // warp, merged in distributed shared memory: one launch, no workspace.
     const int warps = (n_kv_heads > 0 && n_q_heads / n_kv_heads > 8) ? 8 : 16;
     long long cs = (window + 16LL * warps - 1) / (16LL * warps);
-    if (cs > SWA_DECODE_MAX_CLUSTER) cs = SWA_DECODE_MAX_CLUSTER;
+    if (cs > kDecodeMaxCluster) cs = kDecodeMaxCluster;
     if (cs < 1) cs = 1;
     long long cper = (window + cs - 1) / cs;
     cper = (cper + 15) / 16 * 16;
@@ -229,7 +325,7 @@ DecodeSplit decode_split(int batch, int n_q_heads, int n_kv_heads, int window) {
 
 extern "C" {
 
-int swa_abi_version(void) { return 100; }
+int swa_abi_version(void) { return 200; }
 
 const char* swa_last_error(void) { return g_last_error; }
 
@@ -261,48 +357,49 @@ int swa_cache_append(const swa_dims* dims, void* k_cache, void* v_cache, const v
   return ok();
 }
 
+size_t swa_prefill_workspace_size(const swa_dims* dims, int32_t max_tokens) {
+  if (check_dims(dims) != SWA_OK) return 0;
+  if (max_tokens < 1 || max_tokens > dims->window) return 0;
+  const int hpc = swa::prefill_heads_per_cta(dims->n_q_heads, dims->n_kv_heads);
+  return swa::prefill_workspace_bytes(hpc, dims->head_dim);
+}
+
 int swa_prefill_chunk(const swa_dims* dims, void* out, const void* q, const void* k, const void* v,
                       int32_t max_tokens, const void* k_cache, const void* v_cache, const int32_t* start_pos,
-                      const int32_t* n_tokens, void* stream) {
+                      const int32_t* n_tokens, void* workspace, size_t workspace_bytes, void* stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_ptrs("out, q, k, v, k_cache, v_cache", {out, q, k, v, k_cache, v_cache}))) return rc;
   if ((rc = check_int_ptrs("start_pos, n_tokens", {start_pos, n_tokens}))) return rc;
   if (max_tokens < 1 || max_tokens > dims->window)
     return fail(SWA_ERR_INVALID_ARG, "max_tokens %d not in [1, window=%d]", max_tokens, dims->window);
+  if (workspace == nullptr) {
+    if (workspace_bytes != 0)
+      return fail(SWA_ERR_INVALID_ARG, "workspace is NULL but workspace_bytes is %zu", workspace_bytes);
+  } else {
+    if (!aligned16(workspace)) return fail(SWA_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+    const size_t need = swa_prefill_workspace_size(dims, max_tokens);
+    if (workspace_bytes < need)
+      return fail(SWA_ERR_WORKSPACE_TOO_SMALL, "prefill workspace of %zu bytes, %zu needed", workspace_bytes,
+                  need);
+  }
   const int B = dims->batch, Hq = dims->n_q_heads, Hkv = dims->n_kv_heads, D = dims->head_dim;
   const int W = dims->window;
+  const int hpc = swa::prefill_heads_per_cta(Hq, Hkv);
+  const int n_q_tiles = (max_tokens + 127) / 128;
+  const long long n_units = (long long)B * (Hq / hpc) * n_q_tiles;
+  if (n_units > (1LL << 29))
+    return fail(SWA_ERR_UNSUPPORTED, "%lld query tiles x head pairs in one call (limit 2^29)", n_units);
   int* status = nullptr;
   if ((rc = status_ptr(&status))) return rc;
-  EncodeTiledFn enc = nullptr;
-  if ((rc = get_encode(&enc))) return rc;
-
-  int box_d = 0, swz = 0;
-  swa::prefill_map_geometry(D, &box_d, &swz);
+  int device = 0;
+  cudaError_t e = cudaGetDevice(&device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   swa::PrefillMaps maps;
-  memset(&maps, 0, sizeof(maps));
-  const cuuint64_t es = 2;  // bf16
-  {
-    cuuint64_t dims4[4] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)max_tokens, (cuuint64_t)B};
-    cuuint64_t str4[3] = {D * es, (cuuint64_t)Hq * D * es, (cuuint64_t)max_tokens * Hq * D * es};
-    cuuint32_t box4[4] = {(cuuint32_t)box_d, 1, 128, 1};
-    if ((rc = encode_map(enc, &maps.q, q, 4, dims4, str4, box4, swz, "q"))) return rc;
-  }
-  {
-    cuuint64_t dims4[4] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)max_tokens, (cuuint64_t)B};
-    cuuint64_t str4[3] = {D * es, (cuuint64_t)Hkv * D * es, (cuuint64_t)max_tokens * Hkv * D * es};
-    cuuint32_t box4[4] = {(cuuint32_t)box_d, 1, 128, 1};
-    if ((rc = encode_map(enc, &maps.k, k, 4, dims4, str4, box4, swz, "k"))) return rc;
-    if ((rc = encode_map(enc, &maps.v, v, 4, dims4, str4, box4, swz, "v"))) return rc;
-  }
-  {
-    cuuint64_t dims3[3] = {(cuuint64_t)D, (cuuint64_t)W, (cuuint64_t)B * Hkv};
-    cuuint64_t str3[2] = {D * es, (cuuint64_t)W * D * es};
-    cuuint32_t box3[3] = {(cuuint32_t)box_d, 128, 1};
-    if ((rc = encode_map(enc, &maps.kc, k_cache, 3, dims3, str3, box3, swz, "k_cache"))) return rc;
-    if ((rc = encode_map(enc, &maps.vc, v_cache, 3, dims3, str3, box3, swz, "v_cache"))) return rc;
-  }
+  if ((rc = prefill_maps(device, dims, max_tokens, q, k, v, k_cache, v_cache, &maps))) return rc;
 
+  const swa::PrefillSchedule sc =
+      swa::prefill_schedule(n_units, (W + 127) / 128, swa::device_sm_count(device), workspace != nullptr);
   swa::PrefillParams p;
   p.out = out;
   p.start_pos = start_pos;
@@ -314,12 +411,17 @@ int swa_prefill_chunk(const swa_dims* dims, void* out, const void* q, const void
   p.head_dim = D;
   p.window = W;
   p.max_tokens = max_tokens;
-  p.heads_per_cta = ((Hq / Hkv) % 2 == 0) ? 2 : 1;
-  p.n_q_tiles = (max_tokens + 127) / 128;
+  p.heads_per_cta = hpc;
+  p.n_q_tiles = n_q_tiles;
+  p.n_whole = (int)sc.n_whole;
+  p.n_pieces = sc.n_pieces;
+  p.n_items = (int)sc.n_items;
+  p.persistent = sc.persistent;
+  p.workspace = workspace;
   p.scale_log2 = dims->scale * 1.4426950408889634f;
   p.out_f32 = dims->out_dtype == SWA_DTYPE_F32;
   p.trace = g_trace;
-  cudaError_t e = swa::launch_prefill(p, maps, static_cast<cudaStream_t>(stream));
+  e = swa::launch_prefill(p, maps, (int)sc.grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "swa_prefill_chunk launch");
   return ok();
 }

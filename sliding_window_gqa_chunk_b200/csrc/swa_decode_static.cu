@@ -76,7 +76,13 @@ extern "C" SWA_API int swa_decode_static(const swa_dims* dims, void* out, const 
                                          void* stream) {
   int rc = swa::api_check_decode(dims, out, q, k_new, v_new, k_cache, v_cache, pos);
   if (rc) return rc;
-  const size_t need = swa_decode_workspace_size(dims);
+  // The scratch this launch really uses: none when one split covers the window
+  // or a thread-block cluster merges the splits, else one fp32 partial
+  // (d values, max and sum) per (sequence, query head, split).
+  const swa::DecodeSplit sp =
+      swa::decode_split(dims->batch, dims->n_q_heads, dims->n_kv_heads, dims->window);
+  const size_t bh = (size_t)dims->batch * dims->n_q_heads * sp.n_splits;
+  const size_t need = (sp.cluster || sp.n_splits == 1) ? 0 : bh * (dims->head_dim + 2) * sizeof(float);
   if (need > kStaticScratchBytes)
     return swa::api_fail(SWA_ERR_WORKSPACE_TOO_SMALL,
                          "swa_decode_static: these dims need %zu bytes of decode scratch but the "
@@ -87,8 +93,6 @@ extern "C" SWA_API int swa_decode_static(const swa_dims* dims, void* out, const 
   int* status = nullptr;
   if ((rc = swa::api_status_word(&status))) return rc;
 
-  const swa::DecodeSplit sp =
-      swa::decode_split(dims->batch, dims->n_q_heads, dims->n_kv_heads, dims->window);
   swa::DecodeParams p;
   p.out = out;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -99,7 +103,6 @@ extern "C" SWA_API int swa_decode_static(const swa_dims* dims, void* out, const 
   p.k_cache_w = static_cast<__nv_bfloat16*>(k_cache);
   p.v_cache_w = static_cast<__nv_bfloat16*>(v_cache);
   p.pos = pos;
-  const size_t bh = (size_t)dims->batch * dims->n_q_heads * sp.ws_splits;
   p.ws_o = static_cast<float*>(scratch);
   p.ws_ml = static_cast<float*>(scratch) + bh * dims->head_dim;
   p.status = status;

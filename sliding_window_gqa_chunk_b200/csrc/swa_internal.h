@@ -62,10 +62,22 @@ struct PrefillParams {
   int batch, n_q_heads, n_kv_heads, head_dim, window, max_tokens;
   int heads_per_cta;            // 1 or 2 query heads of one kv group per CTA
   int n_q_tiles;                // ceil(max_tokens / 128)
+  int n_whole;                  // work items that are whole units (query tile x head pair x sequence)
+  int n_pieces;                 // pieces per split unit (units n_whole.. are split)
+  int n_items;                  // total work items
+  int persistent;               // 1: CTAs take items from the workspace counter
   float scale_log2;
   int out_f32;
+  void* workspace;              // caller scratch (NULL: no key-range splits)
   int* trace;                   // progress words in host-mapped memory (trace builds only)
 };
+
+// Query heads of one kv group that share a prefill CTA (and its K/V tiles).
+inline int prefill_heads_per_cta(int n_q_heads, int n_kv_heads) {
+  return ((n_q_heads / n_kv_heads) % 2 == 0) ? 2 : 1;
+}
+// Bytes of the prefill workspace for `hpc` heads per CTA and head_dim `d`.
+size_t prefill_workspace_bytes(int hpc, int d);
 
 // TMA descriptors of the prefill, built on the host per call.
 struct PrefillMaps {
@@ -78,7 +90,17 @@ struct PrefillMaps {
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
-cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& maps, cudaStream_t stream);
+// How a prefill launch covers its units: whole units, the split tail, the grid.
+struct PrefillSchedule {
+  long long n_whole;
+  int n_pieces;
+  long long n_items;
+  int persistent;
+  long long grid;
+};
+PrefillSchedule prefill_schedule(long long n_units, int n_wtiles, int n_sms, bool have_workspace);
+int device_sm_count(int device);
+cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& maps, int grid, cudaStream_t stream);
 // TMA box width (elements of d per box row) and swizzle span used by the prefill kernel.
 void prefill_map_geometry(int head_dim, int* box_elems, int* swizzle_bytes);
 

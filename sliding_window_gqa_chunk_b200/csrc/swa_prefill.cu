@@ -68,14 +68,22 @@ constexpr int kThreads = 384;       // 12 warps = 3 warpgroups
 // block's register pool), or setmaxnreg.inc would wait forever; the host
 // refuses to launch if ptxas did not allocate exactly kLaunchRegs.
 constexpr int kLaunchRegs = 168;
-constexpr int kSoftmaxRegs = 224;
-constexpr int kOtherRegs = 56;
+constexpr int kSoftmaxRegs = 208;
+constexpr int kOtherRegs = 88;
 static_assert(2 * kSoftmaxRegs + kOtherRegs == 3 * kLaunchRegs, "register split must fill the pool");
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kVProducerWarp = 10;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
 constexpr uint32_t kTmemCols = 512;
+// Workspace layout: two scheduler counters; one merge counter per split unit
+// and softmax warp (at most one split unit per persistent CTA); then one fp32
+// partial result slot per key-range piece (at most one per persistent CTA):
+// per head, O^T [d][128 rows] followed by the running max [128] and sum [128].
+constexpr int kMaxPersistentCtas = 256;
+constexpr size_t kWsMergeOffset = 256;
+constexpr size_t kWsPartialOffset = 16384;
+static_assert(kWsMergeOffset + kMaxPersistentCtas * 8 * sizeof(int) <= kWsPartialOffset, "workspace layout");
 // Which of every 8 consecutive (even, odd) column pairs take the FMA-pipe
 // exp2 (swa_exp2.cuh) instead of the SFU: bit w set means pair w mod 8.  The
 // SFU's exp2 has a quarter of the FMA pipe's lane rate, so moving a fraction
@@ -85,11 +93,6 @@ constexpr uint32_t kTmemCols = 512;
 #define SWA_EXP2_FMA_PAIRS 0x00
 #endif
 
-// Which of every 8 consecutive (even, odd) column pairs of a fully visible tile
-// take the FMA-pipe exp2 instead of the SFU (bit w set: pair w mod 8).
-#ifndef SWA_EXP2_FMA_PAIRS
-#define SWA_EXP2_FMA_PAIRS 0x00
-#endif
 // K / V ring depths for head_dim 128 (2 Q tiles + K + V must fit in 227 KB).
 #ifndef SWA_K_STAGES_D128
 #define SWA_K_STAGES_D128 3
@@ -193,6 +196,87 @@ __device__ __forceinline__ void store16<__nv_bfloat16>(__nv_bfloat16* dst, const
   }
 }
 
+
+// One work item: a piece of one unit (a 128-row query tile of one sequence and
+// one head pair).  Units are numbered heaviest first: query tile index
+// descending (in a chunk that starts its prompt tile qt sees qt + 1 key
+// tiles), then sequence, then head pair.  Items [0, n_whole) are whole units;
+// the last units are split into n_pieces pieces that take consecutive parts of
+// the unit's key tiles, and their partial softmax results are merged by the
+// piece that finishes last.
+struct Item {
+  int b, qt, kvh, h_first, t_lo;
+  long long s;        // start position of the chunk
+  int n;              // tokens of the sequence in this chunk
+  bool rows;          // the unit has query rows to compute
+  bool bad_args;      // start_pos / n_tokens out of range for this sequence
+  int piece, np;      // piece index and piece count (np == 1: whole unit)
+  int merge_idx;      // split unit index (merge counters)
+  int slot;           // partial result slot of this piece
+  int j0, n_tiles;    // the piece's tiles: plan tiles [j0, j0 + n_tiles)
+  TilePlan plan;
+};
+
+__device__ __forceinline__ Item decode_item(const PrefillParams& p, int item) {
+  Item it;
+  int u;
+  if (item < p.n_whole) {
+    u = item;
+    it.piece = 0;
+    it.np = 1;
+    it.merge_idx = 0;
+    it.slot = 0;
+  } else {
+    const int k = item - p.n_whole;
+    u = p.n_whole + k / p.n_pieces;
+    it.piece = k % p.n_pieces;
+    it.np = p.n_pieces;
+    it.merge_idx = k / p.n_pieces;
+    it.slot = k;
+  }
+  const int hpc = p.heads_per_cta;
+  const int nhp = p.n_q_heads / hpc;
+  const int per_qt = p.batch * nhp;
+  it.qt = p.n_q_tiles - 1 - u / per_qt;
+  const int r = u - (u / per_qt) * per_qt;
+  it.b = r / nhp;
+  const int hp = r - it.b * nhp;
+  const int G = p.n_q_heads / p.n_kv_heads;
+  const int pairs = G / hpc;
+  it.kvh = hp / pairs;
+  it.h_first = it.kvh * G + (hp - it.kvh * pairs) * hpc;
+  it.t_lo = it.qt * kRows;
+  it.s = p.start_pos[it.b];
+  it.n = p.n_tokens[it.b];
+  it.bad_args = it.s < 0 || it.n < 0 || it.n > p.max_tokens;
+  it.rows = !it.bad_args && it.t_lo < it.n;
+  it.j0 = 0;
+  it.n_tiles = 0;
+  it.plan.n_cache = it.plan.first_cache = it.plan.n_chunk = 0;
+  it.plan.n_wtiles = 1;
+  if (it.rows) {
+    it.plan = make_plan(it.s, it.t_lo, it.qt, p.window);
+    const int w = it.plan.total();
+    it.j0 = (int)((long long)it.piece * w / it.np);
+    it.n_tiles = (int)((long long)(it.piece + 1) * w / it.np) - it.j0;
+  }
+  return it;
+}
+
+// Partial result slot of one piece and head: O^T [D][128 rows], then the
+// running max [128] and sum [128] (log2 domain, as the softmax keeps them).
+template <int D>
+__device__ __forceinline__ float* partial_slot(const PrefillParams& p, int slot, int head) {
+  return reinterpret_cast<float*>(static_cast<uint8_t*>(p.workspace) + kWsPartialOffset) +
+         ((size_t)slot * p.heads_per_cta + head) * (size_t)(kRows * (D + 2));
+}
+
+__device__ __forceinline__ float ld_cg(const float* a) {
+  float v;
+  asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(a));
+  return v;
+}
+
 }  // namespace
 
 template <int D, typename OutT>
@@ -205,27 +289,9 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Heaviest query tiles first: in a chunk that starts the prompt, tile qt has
-  // qt + 1 key tiles, so later tiles are dispatched first.
-  const int qt = gridDim.x - 1 - blockIdx.x;
-  const int b = blockIdx.z;
   const int hpc = p.heads_per_cta;
-  const int G = p.n_q_heads / p.n_kv_heads;
-  const int pairs = G / hpc;
-  const int kvh = blockIdx.y / pairs;
-  const int h_first = kvh * G + (blockIdx.y % pairs) * hpc;
   const int W = p.window;
-
-  const long long s = p.start_pos[b];
-  const int n = p.n_tokens[b];
-  if (s < 0 || n < 0 || n > p.max_tokens) {
-    if (threadIdx.x == 0 && qt == 0 && blockIdx.y == 0) raise_status(p.status, SWA_ERR_DEVICE_ARG);
-    return;
-  }
-  const int t_lo = qt * kRows;
-  if (t_lo >= n) return;  // whole CTA: nothing of this sequence in the tile
-  const TilePlan plan = make_plan(s, t_lo, qt, W);
-  const int n_tiles = plan.total();
+  int* const ws_ctr = static_cast<int*>(p.workspace);  // [0] next item, [1] CTAs done
 
   // ---- shared memory carve-up (1024-byte aligned for the 128B swizzle) ----
   const uint32_t raw_addr = tc::smem_u32(smem_raw);
@@ -237,18 +303,27 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
   const uint32_t sBar = base + C::kSmemTiles;
   // barrier addresses (8 bytes each)
   const uint32_t bar_q_full = sBar;
-  const uint32_t bar_k_full = sBar + 8;                // [NK]
+  const uint32_t bar_q_empty = sBar + 8;
+  const uint32_t bar_k_full = sBar + 16;               // [NK]
   const uint32_t bar_k_empty = bar_k_full + 8 * NK;    // [NK]
   const uint32_t bar_v_full = bar_k_empty + 8 * NK;    // [NV]
   const uint32_t bar_v_empty = bar_v_full + 8 * NV;    // [NV]
   const uint32_t bar_s_full = bar_v_empty + 8 * NV;    // [2]
   const uint32_t bar_p_full = bar_s_full + 16;         // [2]
   const uint32_t bar_o_full = bar_p_full + 16;         // [2]
-  const uint32_t bar_done = bar_o_full + 16;
+  const uint32_t bar_item_full = bar_o_full + 16;      // [2]
+  const uint32_t bar_item_empty = bar_item_full + 16;  // [2]
+  const uint32_t bar_done = bar_item_empty + 16;
+  static_assert(16 + 16 * NK + 16 * NV + 6 * 16 + 8 <= 256, "barrier area");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::kSmemTiles + 256);
+  volatile int* item_q = reinterpret_cast<volatile int*>(base_ptr + C::kSmemTiles + 264);  // [2]
+  // Consumers of the item queue: the V producer, the MMA warp and every
+  // softmax warp (one arrival each).
+  const int n_item_consumers = 2 + 4 * hpc;
 
   if (threadIdx.x == 0) {
     tc::mbar_init(bar_q_full, 1);
+    tc::mbar_init(bar_q_empty, 1);
     for (int i = 0; i < NK; ++i) {
       tc::mbar_init(bar_k_full + 8 * i, 1);
       tc::mbar_init(bar_k_empty + 8 * i, 1);
@@ -261,6 +336,8 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
       tc::mbar_init(bar_s_full + 8 * i, 1);
       tc::mbar_init(bar_p_full + 8 * i, kRows / 32);  // one arrival per softmax warp
       tc::mbar_init(bar_o_full + 8 * i, 1);
+      tc::mbar_init(bar_item_full + 8 * i, 1);
+      tc::mbar_init(bar_item_empty + 8 * i, n_item_consumers);
     }
     tc::mbar_init(bar_done, 1);
     tc::mbar_fence_init();
@@ -277,48 +354,81 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) SWA_TRACE_AT(0, 3);
 
+  // Item queue: the K producer fetches items (the CTA's own index first, then
+  // from the shared counter when the grid is persistent) and publishes each in
+  // a two-entry ring; every other role reads the same sequence.  An index
+  // >= n_items ends the sequence.
+  auto next_item = [&](int it, bool& ok) -> int {
+    const int slot = it & 1;
+    ok = tc::mbar_wait(bar_item_full + 8 * slot, (it >> 1) & 1, p.status);
+    const int item = ok ? item_q[slot] : p.n_items;
+    return item;
+  };
+
   // setmaxnreg is per warpgroup and must dominate the code it budgets, so the
   // role dispatch happens inside the two register branches.
   if (warp >= 8) {
   tc::regs_decrease<kOtherRegs>();
   if (warp == kProducerWarp) {
-    // ====================== TMA producer: Q, then K tiles ======================
+    // =============== item fetcher and TMA producer: Q, then K tiles ===============
     if (lane == 0) {
       tc::prefetch_map(&maps.q);
       tc::prefetch_map(&maps.k);
       tc::prefetch_map(&maps.kc);
-      tc::mbar_arrive_expect_tx(bar_q_full, hpc * C::kTileBytes);
-      for (int i = 0; i < hpc; ++i)
-        for (int cb = 0; cb < C::kColBlocks; ++cb)
-          tc::tma_load_4d(sQ + i * C::kTileBytes + cb * C::kBlockBytes, &maps.q, cb * C::kBoxD,
-                          h_first + i, t_lo, b, bar_q_full);
+      int kt = 0;   // K tiles issued (ring position)
+      int qi = 0;   // Q tiles issued (items with tiles)
       bool ok = true;
-      for (int j = 0; j < n_tiles && ok; ++j) {
-        bool is_cache;
-        int kbase;
-        plan.at(j, is_cache, kbase);
-        const int sk = j % NK;
-        SWA_TRACE_AT(1, 1000 + j);
-        if (j >= NK) ok = tc::mbar_wait(bar_k_empty + 8 * sk, ((j / NK) - 1) & 1, p.status);
+      for (int it = 0; ok; ++it) {
+        int item = p.n_items;
+        if (it == 0) item = blockIdx.x;
+        else if (p.persistent) item = (int)gridDim.x + atomicAdd(ws_ctr, 1);
+        const int slot = it & 1;
+        if (it >= 2) ok = tc::mbar_wait(bar_item_empty + 8 * slot, ((it >> 1) - 1) & 1, p.status);
         if (!ok) break;
-        const uint32_t kdst = sK + sk * C::kTileBytes;
-        tc::mbar_arrive_expect_tx(bar_k_full + 8 * sk, C::kTileBytes);
+        if (item > p.n_items) item = p.n_items;
+        item_q[slot] = item;
+        tc::mbar_arrive(bar_item_full + 8 * slot);
+        if (item >= p.n_items) break;
+        const Item I = decode_item(p, item);
+        if (I.bad_args && I.qt == 0 && I.piece == 0 && I.h_first == 0)
+          raise_status(p.status, SWA_ERR_DEVICE_ARG);
+        if (I.n_tiles == 0) continue;
+        SWA_TRACE_AT(1, 1000 + it);
+        if (qi > 0) ok = tc::mbar_wait(bar_q_empty, (qi - 1) & 1, p.status);
+        if (!ok) break;
+        tc::mbar_arrive_expect_tx(bar_q_full, hpc * C::kTileBytes);
+        for (int i = 0; i < hpc; ++i)
+          for (int cb = 0; cb < C::kColBlocks; ++cb)
+            tc::tma_load_4d(sQ + i * C::kTileBytes + cb * C::kBlockBytes, &maps.q, cb * C::kBoxD,
+                            I.h_first + i, I.t_lo, I.b, bar_q_full);
+        ++qi;
+        for (int j = 0; j < I.n_tiles; ++j, ++kt) {
+          bool is_cache;
+          int kbase;
+          I.plan.at(I.j0 + j, is_cache, kbase);
+          const int sk = kt % NK;
+          if (kt >= NK) ok = tc::mbar_wait(bar_k_empty + 8 * sk, ((kt / NK) - 1) & 1, p.status);
+          if (!ok) break;
+          const uint32_t kdst = sK + sk * C::kTileBytes;
+          tc::mbar_arrive_expect_tx(bar_k_full + 8 * sk, C::kTileBytes);
 #ifdef SWA_TILE_COUNTERS
-        if (p.trace != nullptr) atomicAdd(p.trace, 1);  // checked build: key tiles loaded
+          if (p.trace != nullptr) atomicAdd(p.trace, 1);  // checked build: key tiles loaded
 #endif
-        for (int cb = 0; cb < C::kColBlocks; ++cb) {
-          if (is_cache)
-            tc::tma_load_3d(kdst + cb * C::kBlockBytes, &maps.kc, cb * C::kBoxD, kbase,
-                            b * p.n_kv_heads + kvh, bar_k_full + 8 * sk);
-          else
-            tc::tma_load_4d(kdst + cb * C::kBlockBytes, &maps.k, cb * C::kBoxD, kvh, kbase, b,
-                            bar_k_full + 8 * sk);
+          for (int cb = 0; cb < C::kColBlocks; ++cb) {
+            if (is_cache)
+              tc::tma_load_3d(kdst + cb * C::kBlockBytes, &maps.kc, cb * C::kBoxD, kbase,
+                              I.b * p.n_kv_heads + I.kvh, bar_k_full + 8 * sk);
+            else
+              tc::tma_load_4d(kdst + cb * C::kBlockBytes, &maps.k, cb * C::kBoxD, I.kvh, kbase, I.b,
+                              bar_k_full + 8 * sk);
+          }
         }
       }
-      // Before leaving, make sure no copy issued here is still in flight.
+      // Before leaving, make sure no copy issued here is still in flight: the
+      // last Q load and the last use of every K stage.
       SWA_TRACE_AT(1, 5000);
-      tc::mbar_wait(bar_q_full, 0, p.status);
-      for (int j = n_tiles > NK ? n_tiles - NK : 0; j < n_tiles; ++j)
+      if (qi > 0) tc::mbar_wait(bar_q_full, (qi - 1) & 1, p.status);
+      for (int j = kt > NK ? kt - NK : 0; j < kt; ++j)
         tc::mbar_wait(bar_k_full + 8 * (j % NK), (j / NK) & 1, p.status);
       SWA_TRACE_AT(1, 9999);
     }
@@ -329,26 +439,33 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
     if (lane == 0) {
       tc::prefetch_map(&maps.v);
       tc::prefetch_map(&maps.vc);
+      int vt = 0;
       bool ok = true;
-      for (int j = 0; j < n_tiles && ok; ++j) {
-        bool is_cache;
-        int kbase;
-        plan.at(j, is_cache, kbase);
-        const int sv = j % NV;
-        if (j >= NV) ok = tc::mbar_wait(bar_v_empty + 8 * sv, ((j / NV) - 1) & 1, p.status);
-        if (!ok) break;
-        const uint32_t vdst = sV + sv * C::kTileBytes;
-        tc::mbar_arrive_expect_tx(bar_v_full + 8 * sv, C::kTileBytes);
-        for (int cb = 0; cb < C::kColBlocks; ++cb) {
-          if (is_cache)
-            tc::tma_load_3d(vdst + cb * C::kBlockBytes, &maps.vc, cb * C::kBoxD, kbase,
-                            b * p.n_kv_heads + kvh, bar_v_full + 8 * sv);
-          else
-            tc::tma_load_4d(vdst + cb * C::kBlockBytes, &maps.v, cb * C::kBoxD, kvh, kbase, b,
-                            bar_v_full + 8 * sv);
+      for (int it = 0; ok; ++it) {
+        const int item = next_item(it, ok);
+        tc::mbar_arrive(bar_item_empty + 8 * (it & 1));
+        if (!ok || item >= p.n_items) break;
+        const Item I = decode_item(p, item);
+        for (int j = 0; j < I.n_tiles; ++j, ++vt) {
+          bool is_cache;
+          int kbase;
+          I.plan.at(I.j0 + j, is_cache, kbase);
+          const int sv = vt % NV;
+          if (vt >= NV) ok = tc::mbar_wait(bar_v_empty + 8 * sv, ((vt / NV) - 1) & 1, p.status);
+          if (!ok) break;
+          const uint32_t vdst = sV + sv * C::kTileBytes;
+          tc::mbar_arrive_expect_tx(bar_v_full + 8 * sv, C::kTileBytes);
+          for (int cb = 0; cb < C::kColBlocks; ++cb) {
+            if (is_cache)
+              tc::tma_load_3d(vdst + cb * C::kBlockBytes, &maps.vc, cb * C::kBoxD, kbase,
+                              I.b * p.n_kv_heads + I.kvh, bar_v_full + 8 * sv);
+            else
+              tc::tma_load_4d(vdst + cb * C::kBlockBytes, &maps.v, cb * C::kBoxD, I.kvh, kbase, I.b,
+                              bar_v_full + 8 * sv);
+          }
         }
       }
-      for (int j = n_tiles > NV ? n_tiles - NV : 0; j < n_tiles; ++j)
+      for (int j = vt > NV ? vt - NV : 0; j < vt; ++j)
         tc::mbar_wait(bar_v_full + 8 * (j % NV), (j / NV) & 1, p.status);
     }
   } else if (warp == kMmaWarp) {
@@ -388,39 +505,69 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
       };
 
       SWA_TRACE_AT(2, 10);
-      bool ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_q_full, 0, p.status));
-      tc::tc_fence_after();
-      // Per tile j: for each head slot i, O_i += P_i(j-1) V(j-1) (needs the
-      // softmax of tile j-1), then S_i(j) = Q_i K(j)^T.  A tcgen05.commit tracks
-      // every MMA issued before it, so the V stage is released right after the
-      // last PV that reads it and the K stage right after the last S.
-      for (int j = 0; j <= n_tiles && ok; ++j) {
-        const bool has_s = j < n_tiles;
-        const int sk = j % NK;
-        if (has_s) {
-          SWA_TRACE_AT(2, 1000 + j);
-          ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_k_full + 8 * sk, (j / NK) & 1, p.status));
-          if (!ok) break;
+      int kt = 0;   // K tiles consumed
+      int vt = 0;   // V tiles consumed
+      int g0 = 0;   // S tiles before the current item (S / P barrier phases)
+      int qi = 0;   // items with tiles
+      bool ok = true;
+      for (int it = 0; ok; ++it) {
+        int item;
+        {
+          bool got;
+          item = next_item(it, got);
+          ok = __all_sync(0xffffffffu, got);
         }
-        const int svp = (j - 1) % NV;
-        for (int i = 0; i < hpc && ok; ++i) {
-          if (j > 0) {
-            ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_p_full + 8 * i, (j - 1) & 1, p.status));
-            if (ok && i == 0) ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_v_full + 8 * svp, ((j - 1) / NV) & 1, p.status));
-            if (!ok) break;
-            tc::tc_fence_after();
-            issue_pv(i, svp, j - 1 > 0);
-            if (i == hpc - 1) tc::tc_commit_elect(bar_v_empty + 8 * svp);
-            if (!has_s) tc::tc_commit_elect(bar_o_full + 8 * i);
-          }
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(bar_item_empty + 8 * (it & 1));
+        if (!ok || item >= p.n_items) break;
+        const Item I = decode_item(p, item);
+        const int n_tiles = I.n_tiles;
+        if (n_tiles == 0) continue;
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_q_full, qi & 1, p.status));
+        if (!ok) break;
+        ++qi;
+        tc::tc_fence_after();
+        // Per tile j: for each head slot i, O_i += P_i(j-1) V(j-1) (needs the
+        // softmax of tile j-1), then S_i(j) = Q_i K(j)^T.  A tcgen05.commit
+        // tracks every MMA issued before it, so the V stage is released right
+        // after the last PV that reads it, the K stage right after the last S,
+        // and the Q tiles after the item's last S.
+        for (int j = 0; j <= n_tiles && ok; ++j) {
+          const bool has_s = j < n_tiles;
+          const int sk = kt % NK;
           if (has_s) {
-            tc::tc_fence_after();
-            SWA_TRACE_AT(2, 3000 + j * 2 + i);
-            issue_s(i, sk);
-            tc::tc_commit_elect(bar_s_full + 8 * i);
+            SWA_TRACE_AT(2, 1000 + j);
+            ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_k_full + 8 * sk, (kt / NK) & 1, p.status));
+            if (!ok) break;
           }
+          const int svp = vt % NV;
+          for (int i = 0; i < hpc && ok; ++i) {
+            if (j > 0) {
+              ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_p_full + 8 * i, (g0 + j - 1) & 1, p.status));
+              if (ok && i == 0)
+                ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_v_full + 8 * svp, (vt / NV) & 1, p.status));
+              if (!ok) break;
+              tc::tc_fence_after();
+              issue_pv(i, svp, j - 1 > 0);
+              if (i == hpc - 1) tc::tc_commit_elect(bar_v_empty + 8 * svp);
+              if (!has_s) tc::tc_commit_elect(bar_o_full + 8 * i);
+            }
+            if (has_s) {
+              tc::tc_fence_after();
+              SWA_TRACE_AT(2, 3000 + j * 2 + i);
+              issue_s(i, sk);
+              tc::tc_commit_elect(bar_s_full + 8 * i);
+            }
+          }
+          if (!ok) break;
+          if (has_s) {
+            tc::tc_commit_elect(bar_k_empty + 8 * sk);
+            ++kt;
+            if (j == n_tiles - 1) tc::tc_commit_elect(bar_q_empty);
+          }
+          if (j > 0) ++vt;
         }
-        if (ok && has_s) tc::tc_commit_elect(bar_k_empty + 8 * sk);
+        g0 += n_tiles;
       }
       // All MMAs must have finished before the TMEM is released.
       SWA_TRACE_AT(2, 8000);
@@ -435,192 +582,303 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
     // ============================ softmax / epilogue ============================
     const int i = warp / 4;                   // head slot
     const int row = (warp % 4) * 32 + lane;   // query row within the tile = TMEM lane
-    const int t = t_lo + row;                 // chunk row
-    const long long pos_i = s + t;            // absolute query position
     const uint32_t lane_addr = (uint32_t)((warp % 4) * 32) << 16;
     const uint32_t tS = tmem + lane_addr + i * kKeys;
     const uint32_t tO = tmem + lane_addr + 2 * kKeys + i * D;
     const float sl2 = p.scale_log2;
-    // this row's visible cache slots: the cyclic range [a_i, a_i + len_i)
-    long long lo_i = pos_i - W + 1;
-    if (lo_i < 0) lo_i = 0;
-    const int len_i = (int)(s - lo_i);          // <= W - 1; <= 0 means none
-    const int a_i = (int)(lo_i % W);
-
-    float m_run = -CUDART_INF_F;
-    float l_run = 0.f;
+    int g0 = 0;   // S tiles before the current item
+    int oi = 0;   // items with tiles (O barrier phase)
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      if (row == 0) SWA_TRACE_AT(3 + i, 1000 + j);
-      // tcgen05.ld / st / wait are warp-collective (.sync.aligned): every
-      // decision that guards them must be the same on all 32 lanes.
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_s_full + 8 * i, j & 1, p.status));
-      if (!ok) break;
-      tc::tc_fence_after();
-      float sv[kKeys];
+    for (int it = 0; ok; ++it) {
+      int item;
       {
-        float* chunk = sv;
-#pragma unroll
-        for (int c = 0; c < kKeys / 32; ++c)
-          tc::tmem_ld32(tS + c * 32, *reinterpret_cast<float(*)[32]>(chunk + c * 32));
+        bool got;
+        item = next_item(it, got);
+        ok = __all_sync(0xffffffffu, got);
       }
-      tc::tc_wait_ld();
-#pragma unroll
-      for (int c = 0; c < kKeys / 16; ++c) tc::reg_fence16(sv + c * 16);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar_item_empty + 8 * (it & 1));
+      if (!ok || item >= p.n_items) break;
+      const Item I = decode_item(p, item);
+      if (!I.rows) continue;
+      const int n_tiles = I.n_tiles;
+      const int t = I.t_lo + row;               // chunk row
+      const long long s = I.s;
+      const long long pos_i = s + t;            // absolute query position
+      // this row's visible cache slots: the cyclic range [a_i, a_i + len_i)
+      long long lo_i = pos_i - W + 1;
+      if (lo_i < 0) lo_i = 0;
+      const int len_i = (int)(s - lo_i);          // <= W - 1; <= 0 means none
+      const int a_i = (int)(lo_i % W);
 
-      bool is_cache;
-      int kbase;
-      plan.at(j, is_cache, kbase);
-      bool masked = false;  // this row has invisible keys in this tile
-      if (is_cache) {
-        int d0 = kbase - a_i;
-        if (d0 < 0) d0 += W;
-        masked = !((kbase + kKeys <= W) && (len_i > 0) && (d0 + kKeys <= len_i));
-        if (masked) {
-          // slot kbase + k is visible iff it is < W and (kbase + k - a_i) mod W
-          // < len_i, i.e. k < len_i - d0, or W - d0 <= k < W - d0 + len_i
-          const int a_end = len_i - d0, b_lo = W - d0, b_end = W - d0 + len_i;
-          const int r_end = W - kbase;
+      float m_run = -CUDART_INF_F;
+      float l_run = 0.f;
+      for (int j = 0; j < n_tiles; ++j) {
+        if (row == 0) SWA_TRACE_AT(3 + i, 1000 + j);
+        // tcgen05.ld / st / wait are warp-collective (.sync.aligned): every
+        // decision that guards them must be the same on all 32 lanes.
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_s_full + 8 * i, (g0 + j) & 1, p.status));
+        if (!ok) break;
+        tc::tc_fence_after();
+        float sv[kKeys];
+        {
+          float* chunk = sv;
 #pragma unroll
-          for (int k = 0; k < kKeys; ++k) {
-            const bool vis = (k < a_end || (k >= b_lo && k < b_end)) && k < r_end;
-            if (!vis) sv[k] = -CUDART_INF_F;
+          for (int c = 0; c < kKeys / 32; ++c)
+            tc::tmem_ld32(tS + c * 32, *reinterpret_cast<float(*)[32]>(chunk + c * 32));
+        }
+        tc::tc_wait_ld();
+#pragma unroll
+        for (int c = 0; c < kKeys / 16; ++c) tc::reg_fence16(sv + c * 16);
+
+        bool is_cache;
+        int kbase;
+        I.plan.at(I.j0 + j, is_cache, kbase);
+        bool masked = false;  // this row has invisible keys in this tile
+        if (is_cache) {
+          int d0 = kbase - a_i;
+          if (d0 < 0) d0 += W;
+          masked = !((kbase + kKeys <= W) && (len_i > 0) && (d0 + kKeys <= len_i));
+          if (masked) {
+            // slot kbase + k is visible iff it is < W and (kbase + k - a_i) mod W
+            // < len_i, i.e. k < len_i - d0, or W - d0 <= k < W - d0 + len_i
+            const int a_end = len_i - d0, b_lo = W - d0, b_end = W - d0 + len_i;
+            const int r_end = W - kbase;
+#pragma unroll
+            for (int k = 0; k < kKeys; ++k) {
+              const bool vis = (k < a_end || (k >= b_lo && k < b_end)) && k < r_end;
+              if (!vis) sv[k] = -CUDART_INF_F;
+            }
+          }
+        } else {
+          masked = kbase + kKeys - 1 > t;
+          if (masked) {
+#pragma unroll
+            for (int k = 0; k < kKeys; ++k)
+              if (kbase + k > t) sv[k] = -CUDART_INF_F;
           }
         }
-      } else {
-        masked = kbase + kKeys - 1 > t;
-        if (masked) {
-#pragma unroll
-          for (int k = 0; k < kKeys; ++k)
-            if (kbase + k > t) sv[k] = -CUDART_INF_F;
-        }
-      }
 #ifdef SWA_TILE_COUNTERS
-      {  // checked build: (warp, tile) pairs with / without a masked key
-        const bool wm = __any_sync(0xffffffffu, masked);
-        if (lane == 0 && p.trace != nullptr) atomicAdd(p.trace + (wm ? 1 : 2), 1);
-      }
+        {  // checked build: (warp, tile) pairs with / without a masked key
+          const bool wm = __any_sync(0xffffffffu, masked);
+          if (lane == 0 && p.trace != nullptr) atomicAdd(p.trace + (wm ? 1 : 2), 1);
+        }
 #endif
 
-      // P = exp2(scale * log2(e) * s - base) for the whole tile, written over
-      // the first 64 columns of S_i; returns this thread's sum of the fp32 p.
-      // With track_max it also returns the tile's largest raw score (the max
-      // chains run on the ALU pipe, beside the SFU exponentials).
-      auto exp_pass = [&](float base_neg, bool track_max, float& tile_max) -> float {
-        const uint64_t sl2x2 = f2_pack(sl2, sl2);
-        const uint64_t nbx2 = f2_pack(base_neg, base_neg);
-        uint64_t lsum[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-        float m8[8];
+        // P = exp2(scale * log2(e) * s - base) for the whole tile, written over
+        // the first 64 columns of S_i; returns this thread's sum of the fp32 p.
+        // With track_max it also returns the tile's largest raw score (the max
+        // chains run on the ALU pipe, beside the SFU exponentials).
+        auto exp_pass = [&](float base_neg, bool track_max, float& tile_max) -> float {
+          const uint64_t sl2x2 = f2_pack(sl2, sl2);
+          const uint64_t nbx2 = f2_pack(base_neg, base_neg);
+          uint64_t lsum[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+          float m8[8];
 #pragma unroll
-        for (int a = 0; a < 8; ++a) m8[a] = -CUDART_INF_F;
+          for (int a = 0; a < 8; ++a) m8[a] = -CUDART_INF_F;
 #pragma unroll
-        for (int c = 0; c < kKeys / 32; ++c) {
-          uint32_t pw[16];
+          for (int c = 0; c < kKeys / 32; ++c) {
+            uint32_t pw[16];
 #pragma unroll
-          for (int w = 0; w < 16; ++w) {
-            const float s0 = sv[c * 32 + 2 * w], s1 = sv[c * 32 + 2 * w + 1];
-            if (track_max) m8[w % 8] = fmax3(m8[w % 8], s0, s1);
-            const uint64_t x = f2_fma(f2_pack(s0, s1), sl2x2, nbx2);
-            float p0, p1;
-            f2_unpack(x, p0, p1);
-            if ((SWA_EXP2_FMA_PAIRS >> (w % 8)) & 1) {
-              exp2_fma_pipe(p0, p1);
-            } else {
-              p0 = fast_exp2(p0);
-              p1 = fast_exp2(p1);
+            for (int w = 0; w < 16; ++w) {
+              const float s0 = sv[c * 32 + 2 * w], s1 = sv[c * 32 + 2 * w + 1];
+              if (track_max) m8[w % 8] = fmax3(m8[w % 8], s0, s1);
+              const uint64_t x = f2_fma(f2_pack(s0, s1), sl2x2, nbx2);
+              float p0, p1;
+              f2_unpack(x, p0, p1);
+              if ((SWA_EXP2_FMA_PAIRS >> (w % 8)) & 1) {
+                exp2_fma_pipe(p0, p1);
+              } else {
+                p0 = fast_exp2(p0);
+                p1 = fast_exp2(p1);
+              }
+              lsum[w & 1] = f2_add(lsum[w & 1], f2_pack(p0, p1));
+              pw[w] = pack_bf16x2(p0, p1);
             }
-            lsum[w & 1] = f2_add(lsum[w & 1], f2_pack(p0, p1));
-            pw[w] = pack_bf16x2(p0, p1);
+            tc::tmem_st16(tS + c * 16, pw);  // P (bf16 pairs) over the first 64 columns of S_i
           }
-          tc::tmem_st16(tS + c * 16, pw);  // P (bf16 pairs) over the first 64 columns of S_i
-        }
-        if (track_max)
-          tile_max = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-        float a0, a1, b0, b1;
-        f2_unpack(lsum[0], a0, a1);
-        f2_unpack(lsum[1], b0, b1);
-        return (a0 + a1) + (b0 + b1);
-      };
+          if (track_max)
+            tile_max = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+          float a0, a1, b0, b1;
+          f2_unpack(lsum[0], a0, a1);
+          f2_unpack(lsum[1], b0, b1);
+          return (a0 + a1) + (b0 + b1);
+        };
 
-      // Optimistic pass: exponentiate against the running max right away and
-      // check the tile's max afterwards.  Only if some row's max grew by more
-      // than 2^8 (always on a row's first visible tile) is the tile redone
-      // against the new max.  The decisions are warp-uniform because the
-      // TMEM accesses they guard are warp-collective.
-      float part = 0.f;
-      bool exact = __any_sync(0xffffffffu, m_run == -CUDART_INF_F);
-      if (!exact) {
-        float tmax;
-        part = exp_pass(-m_run, true, tmax);
-        exact = __any_sync(0xffffffffu, tmax * sl2 > m_run + kRescaleThreshold);
+        // Optimistic pass: exponentiate against the running max right away and
+        // check the tile's max afterwards.  Only if some row's max grew by more
+        // than 2^8 (always on a row's first visible tile) is the tile redone
+        // against the new max.  The decisions are warp-uniform because the
+        // TMEM accesses they guard are warp-collective.
+        float part = 0.f;
+        bool exact = __any_sync(0xffffffffu, m_run == -CUDART_INF_F);
+        if (!exact) {
+          float tmax;
+          part = exp_pass(-m_run, true, tmax);
+          exact = __any_sync(0xffffffffu, tmax * sl2 > m_run + kRescaleThreshold);
+        }
+        if (exact) {
+          // row maximum: 8 independent 3-input max chains, then a short tree
+          float mx8[8];
+#pragma unroll
+          for (int a = 0; a < 8; ++a) mx8[a] = fmaxf(sv[a], sv[8 + a]);
+#pragma unroll
+          for (int k = 16; k < kKeys; k += 16) {
+#pragma unroll
+            for (int a = 0; a < 8; ++a) mx8[a] = fmax3(mx8[a], sv[k + a], sv[k + 8 + a]);
+          }
+          const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                                 fmaxf(mx8[6], mx8[7]));
+          const float m_new = fmaxf(m_run, mx * sl2);
+          // Rescale only when this row's max grew by more than 2^8; otherwise keep
+          // the stale max (p <= 2^8 stays exact enough in bf16 and fp32).
+          const bool grow = m_new > m_run + kRescaleThreshold;
+          float alpha = 1.f;
+          if (grow) {
+            alpha = fast_exp2(m_run - m_new);  // 0 while nothing was visible yet
+            l_run *= alpha;
+            m_run = m_new;
+          }
+          if (j > 0 && __any_sync(0xffffffffu, grow)) {
+            // O_i holds this item's previous tiles (its last PV finished before
+            // S_i(j) did).  The whole warp takes this branch; rows that keep
+            // their max multiply by 1.
+#pragma unroll
+            for (int c = 0; c < D / 16; ++c) {
+              float ov[16];
+              tc::tmem_ld16(tO + c * 16, ov);
+              tc::tc_wait_ld();
+              tc::reg_fence16(ov);
+              uint32_t ow[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) ow[e] = __float_as_uint(ov[e] * alpha);
+              tc::tmem_st16(tO + c * 16, ow);
+            }
+          }
+          float unused;
+          part = exp_pass((m_run == -CUDART_INF_F) ? 0.f : -m_run, false, unused);
+        }
+        l_run += part;
+        tc::tc_wait_st();
+        tc::tc_fence_before();
+        __syncwarp();
+#ifdef SWA_TEST_FAULTS
+        // Checked build for the timeout test: with the fault switch on, softmax
+        // warp 0 withholds its P-ready arrival on the last tile of its first
+        // item, so the MMA warp's bounded wait runs out.  No copy is withheld.
+        const bool withhold = p.trace != nullptr && *p.trace == 1 && warp == 0 && it == 0 &&
+                              j == n_tiles - 1;
+        if (lane == 0 && !withhold) tc::mbar_arrive(bar_p_full + 8 * i);
+#else
+        if (lane == 0) tc::mbar_arrive(bar_p_full + 8 * i);
+#endif
+        if (row == 0) SWA_TRACE_AT(3 + i, 2000 + j);
       }
-      if (exact) {
-        // row maximum: 8 independent 3-input max chains, then a short tree
-        float mx8[8];
+      if (!ok) break;
+      g0 += n_tiles;
+
+      // ---------------------------------- epilogue ----------------------------------
+      if (row == 0) SWA_TRACE_AT(3 + i, 7000);
+      const bool have_o = n_tiles > 0;
+      if (have_o) {
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_o_full + 8 * i, oi & 1, p.status));
+        ++oi;
+        if (!ok) break;
+        tc::tc_fence_after();
+      }
+      OutT* dst = reinterpret_cast<OutT*>(p.out) +
+                  (((size_t)I.b * p.max_tokens + t) * p.n_q_heads + (I.h_first + i)) * D;
+      if (I.np == 1) {
+        const float inv_l = 1.f / l_run;
 #pragma unroll
-        for (int a = 0; a < 8; ++a) mx8[a] = fmaxf(sv[a], sv[8 + a]);
-#pragma unroll
-        for (int k = 16; k < kKeys; k += 16) {
-#pragma unroll
-          for (int a = 0; a < 8; ++a) mx8[a] = fmax3(mx8[a], sv[k + a], sv[k + 8 + a]);
+        for (int c = 0; c < D / 16; ++c) {
+          float ov[16];
+          tc::tmem_ld16(tO + c * 16, ov);
+          tc::tc_wait_ld();
+          tc::reg_fence16(ov);
+          if (t < I.n) store16<OutT>(dst + c * 16, ov, inv_l);
         }
-        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                               fmaxf(mx8[6], mx8[7]));
-        const float m_new = fmaxf(m_run, mx * sl2);
-        // Rescale only when this row's max grew by more than 2^8; otherwise keep
-        // the stale max (p <= 2^8 stays exact enough in bf16 and fp32).
-        const bool grow = m_new > m_run + kRescaleThreshold;
-        float alpha = 1.f;
-        if (grow) {
-          alpha = fast_exp2(m_run - m_new);  // 0 while nothing was visible yet
-          l_run *= alpha;
-          m_run = m_new;
-        }
-        if (j > 0 && __any_sync(0xffffffffu, grow)) {
-          // O_i holds the previous tiles' sum (its last PV finished before S_i(j)
-          // did).  The whole warp takes this branch; rows that keep their max
-          // multiply by 1.
+        continue;
+      }
+      // A piece of a split unit: publish this warp's 32 rows of (O, max, sum),
+      // then count the pieces that have done so; the warp that completes the
+      // count merges every piece's rows (its own straight from TMEM) and
+      // writes the output.  Each warp merges its own rows, so warps never wait
+      // for one another.
+      const float m_own = have_o ? m_run : -CUDART_INF_F;
+      const float l_own = have_o ? l_run : 0.f;
+      {
+        float* part = partial_slot<D>(p, I.slot, i);
 #pragma unroll
-          for (int c = 0; c < D / 16; ++c) {
-            float ov[16];
+        for (int c = 0; c < D / 16; ++c) {
+          float ov[16];
+          if (have_o) {
             tc::tmem_ld16(tO + c * 16, ov);
             tc::tc_wait_ld();
             tc::reg_fence16(ov);
-            uint32_t ow[16];
+          } else {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) ow[e] = __float_as_uint(ov[e] * alpha);
-            tc::tmem_st16(tO + c * 16, ow);
+            for (int e = 0; e < 16; ++e) ov[e] = 0.f;
           }
+#pragma unroll
+          for (int e = 0; e < 16; ++e) part[(c * 16 + e) * kRows + row] = ov[e];
         }
-        float unused;
-        part = exp_pass((m_run == -CUDART_INF_F) ? 0.f : -m_run, false, unused);
+        part[D * kRows + row] = m_own;
+        part[D * kRows + kRows + row] = l_own;
       }
-      l_run += part;
-      (void)masked;
-      tc::tc_wait_st();
-      tc::tc_fence_before();
+      __threadfence();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar_p_full + 8 * i);
-      if (row == 0) SWA_TRACE_AT(3 + i, 2000 + j);
-    }
-
-    if (row == 0) SWA_TRACE_AT(3 + i, 7000);
-    if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_o_full + 8 * i, 0, p.status));
-    if (row == 0) SWA_TRACE_AT(3 + i, ok ? 8000 : 7500);
-    if (ok) {
-      tc::tc_fence_after();
-      const float inv_l = 1.f / l_run;
-      OutT* dst = reinterpret_cast<OutT*>(p.out) +
-                  (((size_t)b * p.max_tokens + t) * p.n_q_heads + (h_first + i)) * D;
+      int last = 0;
+      if (lane == 0) {
+        int* ctr = reinterpret_cast<int*>(static_cast<uint8_t*>(p.workspace) + kWsMergeOffset) +
+                   I.merge_idx * 8 + (warp & 7);
+        const int old = atomicAdd(ctr, 1);
+        last = old == I.np - 1;
+        if (last) atomicExch(ctr, 0);  // leave the counter zero for the next call
+      }
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (!last) continue;
+      __threadfence();
+      const int slot0 = I.slot - I.piece;
+      float M = m_own;
+      for (int q = 0; q < I.np; ++q)
+        if (q != I.piece) M = fmaxf(M, ld_cg(partial_slot<D>(p, slot0 + q, i) + D * kRows + row));
+      float a_own = (m_own == -CUDART_INF_F) ? 0.f : fast_exp2(m_own - M);
+      float L = a_own * l_own;
+      float a_q[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        a_q[q] = 0.f;
+        if (q < I.np && q != I.piece) {
+          const float* pq = partial_slot<D>(p, slot0 + q, i);
+          const float mq = ld_cg(pq + D * kRows + row);
+          a_q[q] = (mq == -CUDART_INF_F) ? 0.f : fast_exp2(mq - M);
+          L += a_q[q] * ld_cg(pq + D * kRows + kRows + row);
+        }
+      }
+      const float inv_l = 1.f / L;
 #pragma unroll
       for (int c = 0; c < D / 16; ++c) {
         float ov[16];
-        tc::tmem_ld16(tO + c * 16, ov);
-        tc::tc_wait_ld();
-        tc::reg_fence16(ov);
-        if (t < n) store16<OutT>(dst + c * 16, ov, inv_l);
+        if (have_o) {
+          tc::tmem_ld16(tO + c * 16, ov);
+          tc::tc_wait_ld();
+          tc::reg_fence16(ov);
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) ov[e] = have_o ? ov[e] * a_own : 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (q < I.np && q != I.piece && a_q[q] != 0.f) {
+            const float* pq = partial_slot<D>(p, slot0 + q, i) + (c * 16) * kRows + row;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) ov[e] += a_q[q] * ld_cg(pq + e * kRows);
+          }
+        }
+        if (t < I.n) store16<OutT>(dst + c * 16, ov, inv_l);
       }
     }
+    if (row == 0) SWA_TRACE_AT(3 + i, ok ? 8000 : 7500);
   }
   }
 
@@ -633,12 +891,27 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
     tc::tmem_dealloc(tmem, kTmemCols);
     if (lane == 0) SWA_TRACE_AT(5, 3);
   }
+  if (threadIdx.x == 0 && p.persistent) {
+    // The last CTA to finish resets the scheduler counters for the next call
+    // (every CTA has made its last fetch before it gets here).
+    __threadfence();
+    if (atomicAdd(ws_ctr + 1, 1) == (int)gridDim.x - 1) {
+      atomicExch(ws_ctr, 0);
+      atomicExch(ws_ctr + 1, 0);
+    }
+  }
 }
 
 namespace {
 
+// Per device: SM count, and which kernel instantiations had their dynamic
+// shared memory limit raised (set once per device, not per launch).
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices] = {};
+
 template <int D, typename OutT>
-cudaError_t launch_prefill_t(const PrefillParams& p, const PrefillMaps& maps, cudaStream_t stream) {
+cudaError_t launch_prefill_t(const PrefillParams& p, const PrefillMaps& maps, int grid, int device,
+                             cudaStream_t stream) {
   using C = Cfg<D>;
   auto kern = swa_prefill_kernel<D, OutT>;
   // The setmaxnreg split assumes the launch register count; never launch with another.
@@ -650,24 +923,32 @@ cudaError_t launch_prefill_t(const PrefillParams& p, const PrefillMaps& maps, cu
     regs = attr.numRegs;
   }
   if (regs != kLaunchRegs) return cudaErrorInvalidKernelImage;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-  if (e != cudaSuccess) return e;
-  dim3 grid(p.n_q_tiles, p.n_q_heads / p.heads_per_cta, p.batch);
+  static bool smem_set[kMaxDevices] = {};
+  if (!smem_set[device]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    smem_set[device] = true;
+  }
   kern<<<grid, kThreads, C::kSmemBytes, stream>>>(p, maps);
   return cudaGetLastError();
 }
 
 template <typename OutT>
-cudaError_t launch_prefill_o(const PrefillParams& p, const PrefillMaps& maps, cudaStream_t stream) {
+cudaError_t launch_prefill_o(const PrefillParams& p, const PrefillMaps& maps, int grid, int device,
+                             cudaStream_t stream) {
   switch (p.head_dim) {
-    case 16: return launch_prefill_t<16, OutT>(p, maps, stream);
-    case 64: return launch_prefill_t<64, OutT>(p, maps, stream);
-    case 128: return launch_prefill_t<128, OutT>(p, maps, stream);
+    case 16: return launch_prefill_t<16, OutT>(p, maps, grid, device, stream);
+    case 64: return launch_prefill_t<64, OutT>(p, maps, grid, device, stream);
+    case 128: return launch_prefill_t<128, OutT>(p, maps, grid, device, stream);
   }
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
+
+size_t prefill_workspace_bytes(int hpc, int d) {
+  return kWsPartialOffset + (size_t)kMaxPersistentCtas * hpc * kRows * (d + 2) * sizeof(float);
+}
 
 void prefill_map_geometry(int head_dim, int* box_elems, int* swizzle_bytes) {
   const int swz = (head_dim * 2 >= 128) ? 128 : head_dim * 2;
@@ -675,9 +956,58 @@ void prefill_map_geometry(int head_dim, int* box_elems, int* swizzle_bytes) {
   *box_elems = swz / 2;
 }
 
-cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& maps, cudaStream_t stream) {
-  if (p.out_f32) return launch_prefill_o<float>(p, maps, stream);
-  return launch_prefill_o<__nv_bfloat16>(p, maps, stream);
+PrefillSchedule prefill_schedule(long long n_units, int n_wtiles, int n_sms, bool have_workspace) {
+  PrefillSchedule sc;
+  sc.n_whole = n_units;
+  sc.n_pieces = 1;
+  sc.n_items = n_units;
+  sc.persistent = 0;
+  sc.grid = n_units;
+  if (!have_workspace || n_units < 1) return sc;
+  long long ctas = n_sms < kMaxPersistentCtas ? n_sms : kMaxPersistentCtas;
+  if (ctas < 1) ctas = 1;
+  // Units are taken heaviest first, so the last round over the SMs is the one
+  // that can leave SMs idle (with fewer units than SMs, the only round).  Its
+  // units (the last `tail` in the order) are cut into pieces of their key
+  // range so that the round fills the SMs: at most ctas pieces in all, at most
+  // 4 per unit, about 4 or more key tiles each for a unit that sees a whole
+  // window (n_wtiles + 1 tiles).
+  const long long tail = n_units % ctas;
+  long long pieces = 1;
+  if (tail > 0) {
+    pieces = ctas / tail;
+    if (pieces > 4) pieces = 4;
+    const long long by_size = (n_wtiles + 1) / 4;
+    if (pieces > by_size) pieces = by_size;
+    if (pieces < 1) pieces = 1;
+  }
+  if (pieces > 1) {
+    sc.n_whole = n_units - tail;
+    sc.n_pieces = (int)pieces;
+  }
+  sc.n_items = sc.n_whole + (n_units - sc.n_whole) * sc.n_pieces;
+  sc.persistent = 1;
+  sc.grid = ctas < sc.n_items ? ctas : sc.n_items;
+  return sc;
+}
+
+cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& maps, int grid, cudaStream_t stream) {
+  int device = 0;
+  cudaError_t e = cudaGetDevice(&device);
+  if (e != cudaSuccess) return e;
+  if (device < 0 || device >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (p.out_f32) return launch_prefill_o<float>(p, maps, grid, device, stream);
+  return launch_prefill_o<__nv_bfloat16>(p, maps, grid, device, stream);
+}
+
+int device_sm_count(int device) {
+  if (device < 0 || device >= kMaxDevices) return 0;
+  if (g_sm_count[device] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return 0;
+    g_sm_count[device] = n;
+  }
+  return g_sm_count[device];
 }
 
 }  // namespace swa

@@ -46,11 +46,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Cycle limit of every bounded wait: about two seconds of SM clock.  Checked
+// builds for the timeout test lower it to about a millisecond.
+#ifndef SWA_WAIT_LIMIT_CYCLES
+#define SWA_WAIT_LIMIT_CYCLES 4000000000LL
+#endif
+
 // Wait for the phase with the given parity to complete.  Gives up after
-// `limit_cycles` SM clock cycles (about two seconds at the default), records
-// SWA_ERR_TIMEOUT in the status word and returns false.
+// `limit_cycles` SM clock cycles, records SWA_ERR_TIMEOUT in the status word
+// and returns false.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* status,
-                                          long long limit_cycles = 4000000000LL) {
+                                          long long limit_cycles = SWA_WAIT_LIMIT_CYCLES) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {

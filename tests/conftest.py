@@ -26,3 +26,17 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    # Measured errors of the GPU parity comparisons (tests/gpu_helpers.assert_close).
+    try:
+        from tests import gpu_helpers
+    except Exception:  # the GPU helpers need the library; nothing was measured then
+        return
+    if not gpu_helpers.MEASURED:
+        return
+    tr = terminalreporter
+    tr.section("parity: measured errors against the oracle")
+    for what, mx, rl, bar in gpu_helpers.MEASURED:
+        tr.write_line(f"{what:60s} max_abs={mx:.3e} rel_l1={rl:.3e} (bar 1e-2 / {bar:.0e})")

@@ -15,6 +15,11 @@ MAX_ABS = 1e-2
 REL_L1 = 2e-3
 REL_L1_BF16_OUT = 4e-3
 
+# (what, max_abs, rel_l1, bar) of every comparison made in this session; the
+# conftest prints them at the end of the run so the measured errors are on
+# record next to the pass/fail verdict.
+MEASURED = []
+
 
 def rel_l1(got, ref):
     got = np.asarray(got, dtype=np.float64)
@@ -31,6 +36,7 @@ def assert_close(got, ref, what="", bf16_out=False):
     mx = float(err.max()) if err.size else 0.0
     rl = rel_l1(got, ref)
     bar = REL_L1_BF16_OUT if bf16_out else REL_L1
+    MEASURED.append((what, mx, rl, bar))
     assert mx <= MAX_ABS and rl <= bar, f"{what}: max_abs={mx:.3e} rel_l1={rl:.3e}"
     return mx, rl
 
@@ -39,11 +45,13 @@ def dev_i32(values, device="cuda"):
     return torch.tensor([int(x) for x in values], dtype=torch.int32, device=device)
 
 
-def gpu_chunked_prefill(dims, q, k, v, lengths, chunk, device="cuda"):
+def gpu_chunked_prefill(dims, q, k, v, lengths, chunk, device="cuda", workspace=True):
     """Prefill padded prompts q/k/v [B, L, H, d] (bf16, CPU) chunk by chunk on
-    the GPU.  Returns (out [B, L, Hq, d] float64 numpy, k_cache, v_cache)."""
+    the GPU (with a prefill workspace, i.e. the persistent split schedule, or
+    without one).  Returns (out [B, L, Hq, d] float64 numpy, k_cache, v_cache)."""
     B, L, Hq, d = q.shape
     kc, vc = swa.new_cache(dims, device)
+    ws = swa.prefill_workspace(dims, chunk, device) if workspace else None
     out = torch.zeros((B, L, Hq, d), dtype=torch.float64)
     n_calls = max((n + chunk - 1) // chunk for n in lengths)
     for c in range(n_calls):
@@ -61,7 +69,7 @@ def gpu_chunked_prefill(dims, q, k, v, lengths, chunk, device="cuda"):
         o = torch.zeros((B, T, Hq, d), dtype=dims.torch_out_dtype, device=device)
         sp = dev_i32([st] * B, device)
         nt = dev_i32(counts, device)
-        swa.prefill_chunk(dims, o, qg, kg, vg, kc, vc, sp, nt)
+        swa.prefill_chunk(dims, o, qg, kg, vg, kc, vc, sp, nt, workspace=ws)
         swa.cache_append(dims, kc, vc, kg, vg, sp, nt)
         out[:, st:hi] = o[:, : hi - st].double().cpu()
     torch.cuda.synchronize()

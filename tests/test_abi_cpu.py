@@ -29,7 +29,8 @@ def declared_symbols():
 
 def test_header_declares_the_boundary():
     names = set(declared_symbols())
-    assert {"swa_cache_append", "swa_prefill_chunk", "swa_decode", "swa_decode_workspace_size",
+    assert {"swa_cache_append", "swa_prefill_chunk", "swa_prefill_workspace_size", "swa_decode",
+            "swa_decode_workspace_size",
             "swa_last_error", "swa_device_status", "swa_abi_version"} <= names
 
 
@@ -39,7 +40,23 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version(lib):
-    assert swa.abi_version() == 100
+    assert swa.abi_version() == 200
+
+
+def test_prefill_workspace_checks(lib):
+    d = dims()
+    need = lib.swa_prefill_workspace_size(ctypes.byref(d), 128)
+    assert need > 0
+    assert lib.swa_prefill_workspace_size(ctypes.byref(d), 0) == 0
+    assert lib.swa_prefill_workspace_size(ctypes.byref(d), 257) == 0
+    p6 = [P()] * 6
+    rc = lib.swa_prefill_chunk(ctypes.byref(d), *p6[:4], 128, *p6[4:], P(), P(), P(), need - 1, None)
+    assert rc == swa.SWA_ERR_WORKSPACE_TOO_SMALL
+    rc = lib.swa_prefill_chunk(ctypes.byref(d), *p6[:4], 128, *p6[4:], P(), P(), P(FAKE + 8), need,
+                               None)
+    assert rc == swa.SWA_ERR_INVALID_ARG and b"workspace" in lib.swa_last_error()
+    rc = lib.swa_prefill_chunk(ctypes.byref(d), *p6[:4], 128, *p6[4:], P(), P(), None, 64, None)
+    assert rc == swa.SWA_ERR_INVALID_ARG
 
 
 def dims(**kw):
@@ -56,7 +73,7 @@ def P(x=FAKE):
 def prefill(lib, d, max_tokens=128, ptrs=None):
     p = ptrs or [P()] * 6
     return lib.swa_prefill_chunk(ctypes.byref(d), p[0], p[1], p[2], p[3], max_tokens, p[4], p[5],
-                                 P(), P(), None)
+                                 P(), P(), None, 0, None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -94,9 +111,9 @@ def test_null_and_misaligned_pointers(lib):
         assert prefill(lib, d, ptrs=ptrs) == swa.SWA_ERR_INVALID_ARG
         assert b"aligned" in lib.swa_last_error()
     assert lib.swa_prefill_chunk(ctypes.byref(d), P(), P(), P(), P(), 16, P(), P(), None, P(),
-                                 None) == swa.SWA_ERR_INVALID_ARG
+                                 None, 0, None) == swa.SWA_ERR_INVALID_ARG
     assert lib.swa_prefill_chunk(None, P(), P(), P(), P(), 16, P(), P(), P(), P(),
-                                 None) == swa.SWA_ERR_INVALID_ARG
+                                 None, 0, None) == swa.SWA_ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("max_tokens", [0, -3, 257])

@@ -9,7 +9,8 @@
 * Receptive field of stacked layers (section 2, Sliding Window Attention and
   Figure 1): with Q = 0 every visible key gets the same weight, so with
   positive values a change at token t reaches exactly positions
-  t .. t + k(W - 1) after k layers.
+  t .. t + k(W - 1) after k layers.  Every chained layer is also compared with
+  the oracle's full-KV windowed attention of its input.
 """
 import numpy as np
 import pytest
@@ -51,7 +52,8 @@ def test_mixed_prefill_and_decode_in_one_launch():
         o = torch.zeros((B, T, Hq, d), dtype=torch.float32, device=DEV)
         sp, nt = dev_i32(starts), dev_i32(counts)
         kg, vg = kcn.to(DEV), vcn.to(DEV)
-        swa.prefill_chunk(dims, o, qc.to(DEV), kg, vg, kc, vc, sp, nt)
+        swa.prefill_chunk(dims, o, qc.to(DEV), kg, vg, kc, vc, sp, nt,
+                          workspace=swa.prefill_workspace(dims, T, DEV))
         swa.cache_append(dims, kc, vc, kg, vg, sp, nt)
         expect = oracle.prefill_chunk(ref, qc, kcn, vcn, starts, counts, dims.scale)
         oracle.cache_append(ref, kcn, vcn, starts, counts)
@@ -98,9 +100,18 @@ def test_receptive_field_of_stacked_layers(k_layers):
     pert = base.clone()
     pert[0, t] = 2.0
     xb, xp = base, pert
-    for _ in range(k_layers):
-        xb = _layer(xb, W).to(torch.bfloat16)
-        xp = _layer(xp, W).to(torch.bfloat16)
+    for layer in range(k_layers):
+        # each chained GPU layer against the oracle's full-KV windowed attention
+        # of that layer's (bf16) input, with Q = 0 as on the GPU
+        for name, x in (("base", xb), ("perturbed", xp)):
+            got = _layer(x, W)
+            ref = oracle.full_kv_banded(torch.zeros_like(x), x, x, W, 1.0)
+            assert_close(got.double().numpy(), ref, f"stacked layer {layer + 1} ({name})")
+            if name == "base":
+                xb_next = got.to(torch.bfloat16)
+            else:
+                xp_next = got.to(torch.bfloat16)
+        xb, xp = xb_next, xp_next
     diff = (xp.float() - xb.float()).abs().amax(dim=(0, 2, 3)).numpy()
     changed = set(np.nonzero(diff > 1e-3)[0].tolist())
     reach = k_layers * (W - 1)

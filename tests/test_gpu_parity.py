@@ -62,11 +62,12 @@ def test_tiny_workload_prefill_then_decode(out_dtype):
     kc, vc = swa.new_cache(dims, DEV)
     ref = oracle.RollingCache(1, s.n_kv_heads, s.window, s.head_dim)
     bf = out_dtype == "bf16"
+    pws = swa.prefill_workspace(dims, 4, DEV)
     for c, (q, k, v) in enumerate(chunks):
         st = 4 * c
         o = torch.zeros((1, 4, s.n_q_heads, s.head_dim), dtype=dims.torch_out_dtype, device=DEV)
         sp, nt = dev_i32([st]), dev_i32([4])
-        swa.prefill_chunk(dims, o, q.to(DEV), k.to(DEV), v.to(DEV), kc, vc, sp, nt)
+        swa.prefill_chunk(dims, o, q.to(DEV), k.to(DEV), v.to(DEV), kc, vc, sp, nt, workspace=pws)
         swa.cache_append(dims, kc, vc, k.to(DEV), v.to(DEV), sp, nt)
         expect = oracle.prefill_chunk(ref, q, k, v, [st], [4], dims.scale)
         oracle.cache_append(ref, k, v, [st], [4])
@@ -128,12 +129,13 @@ PREFILL_CASES = [
 ]
 
 
+@pytest.mark.parametrize("workspace", [True, False], ids=["persistent", "grid"])
 @pytest.mark.parametrize("B,lengths,W,chunk,Hq,Hkv,d", PREFILL_CASES)
-def test_prefill_matches_oracle(B, lengths, W, chunk, Hq, Hkv, d):
+def test_prefill_matches_oracle(B, lengths, W, chunk, Hq, Hkv, d, workspace):
     L = max(lengths)
     q, k, v = random_case(1000 + W + chunk + d, B, L, Hq, Hkv, d, lengths=lengths)
     dims = mk_dims(B, Hq, Hkv, d, W)
-    got, kc, vc = gpu_chunked_prefill(dims, q, k, v, lengths, chunk)
+    got, kc, vc = gpu_chunked_prefill(dims, q, k, v, lengths, chunk, workspace=workspace)
     ref, rcache = oracle.run_chunked_prefill(q, k, v, W, chunk, dims.scale, lengths=lengths)
     assert_close(got, ref, f"prefill B={B} L={lengths} W={W} chunk={chunk}")
     np.testing.assert_array_equal(cache_as_f64(kc), rcache.k)
@@ -169,7 +171,8 @@ def test_prefill_chunk_after_decode_steps():
     o = torch.zeros((B, T, Hq, d), dtype=torch.float32, device=DEV)
     qc, kcn, vcn = (x[:, first:].contiguous() for x in (q, k, v))
     sp, nt = dev_i32([first] * B), dev_i32([T, T - 50])
-    swa.prefill_chunk(dims, o, qc.to(DEV), kcn.to(DEV), vcn.to(DEV), kc, vc, sp, nt)
+    swa.prefill_chunk(dims, o, qc.to(DEV), kcn.to(DEV), vcn.to(DEV), kc, vc, sp, nt,
+                      workspace=swa.prefill_workspace(dims, T, DEV))
     swa.cache_append(dims, kc, vc, kcn.to(DEV), vcn.to(DEV), sp, nt)
     expect = oracle.prefill_chunk(ref, qc, kcn, vcn, [first] * B, [T, T - 50], dims.scale)
     oracle.cache_append(ref, kcn, vcn, [first] * B, [T, T - 50])

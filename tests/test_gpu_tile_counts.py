@@ -36,7 +36,7 @@ def counting_lib():
     lib = ctypes.CDLL(so)
     P, I32 = ctypes.c_void_p, ctypes.c_int32
     D = ctypes.POINTER(swa._CDims)
-    lib.swa_prefill_chunk.argtypes = [D, P, P, P, P, I32, P, P, P, P, P]
+    lib.swa_prefill_chunk.argtypes = [D, P, P, P, P, I32, P, P, P, P, P, ctypes.c_size_t, P]
     lib.swa_prefill_chunk.restype = ctypes.c_int
     lib.swa_device_status.argtypes = [P]
     lib.swa_device_status.restype = ctypes.c_int
@@ -114,7 +114,7 @@ def test_tile_classes_match_brute_force(counting_lib, s, n, T, W, Hq, Hkv):
     try:
         rc = counting_lib.swa_prefill_chunk(
             ctypes.byref(cd), out.data_ptr(), q.data_ptr(), k.data_ptr(), v.data_ptr(), T,
-            kc.data_ptr(), vc.data_ptr(), sp.data_ptr(), nt.data_ptr(), None)
+            kc.data_ptr(), vc.data_ptr(), sp.data_ptr(), nt.data_ptr(), None, 0, None)
         assert rc == 0
         torch.cuda.synchronize()
     finally:
