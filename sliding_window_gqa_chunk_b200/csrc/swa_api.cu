@@ -7,6 +7,7 @@
 // error has enqueued nothing.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cmath>
 #include <cstdarg>
@@ -21,6 +22,14 @@
 namespace {
 
 thread_local char g_last_error[512] = "";
+
+// An NVTX range around each entry point, so profilers (nsys, ncu's NVTX
+// filters) see the library's calls by name.  Header-only NVTX: without a
+// profiler attached a push / pop is a check of a null function pointer.
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+};
 
 int fail(int code, const char* fmt, ...) {
   va_list ap;
@@ -258,17 +267,11 @@ extern "C" SWA_API void swa_debug_set_trace(void* host_mapped) { g_trace = stati
 
 namespace swa {
 
-// Largest thread-block cluster of the decode's split merge (the portable limit).
-constexpr int kDecodeMaxCluster = 8;
 // Non-zero: the number of splits rounds down (at least this many), so that the
 // CTAs fit in one wave of resident 4-warp CTAs (a second, nearly empty wave
 // cost up to a third of the sweep); 0: rounds up.
 #ifndef SWA_DECODE_SPLIT_FLOOR
 #define SWA_DECODE_SPLIT_FLOOR 1
-#endif
-// 0: never merge splits in a cluster (always the workspace and the combine kernel)
-#ifndef SWA_DECODE_CLUSTER
-#define SWA_DECODE_CLUSTER 1
 #endif
 
 DecodeSplit decode_split(int batch, int n_q_heads, int n_kv_heads, int window) {
@@ -290,6 +293,7 @@ DecodeSplit decode_split(int batch, int n_q_heads, int n_kv_heads, int window) {
   s.ws_splits = s.n_splits;
   s.warps = 4;
   s.cluster = 0;
+  s.stream = 0;
 #if SWA_DECODE_SPLIT_FLOOR
   {
     long long fs = target / units;
@@ -302,21 +306,27 @@ DecodeSplit decode_split(int batch, int n_q_heads, int n_kv_heads, int window) {
     s.n_splits = (int)((window + fper - 1) / fper);
   }
 #endif
-  if (SWA_DECODE_CLUSTER && units < 64) {
-    // Few (sequence, kv head) pairs: the sweep is latency-bound, so each pair
-    // gets one cluster of up to 8 CTAs of 16 warps (8 for groups above 8
-    // heads, which need more registers), at least one 16-slot block per
-    // warp, merged in distributed shared memory: one launch, no workspace.
-    const int warps = (n_kv_heads > 0 && n_q_heads / n_kv_heads > 8) ? 8 : 16;
-    long long cs = (window + 16LL * warps - 1) / (16LL * warps);
-    if (cs > kDecodeMaxCluster) cs = kDecodeMaxCluster;
-    if (cs < 1) cs = 1;
+  if (units < 148) {
+    // Fewer (sequence, kv head) pairs than SMs: one launch of CTAs whose
+    // producer warp streams the split's slots into shared memory with bulk
+    // copies, so every byte of a split is in flight at once.  Below 64 pairs
+    // the window of a pair is split over a thread-block cluster of up to 8
+    // CTAs (about 512 slots each) that merge through distributed shared
+    // memory; from 64 pairs on one CTA covers a pair's whole window.  No
+    // workspace and no combine kernel either way.
+    long long cs = 1;
+    if (units < 64) {
+      cs = (window + 511) / 512;
+      if (cs > kDecodeMaxClusterSplits) cs = kDecodeMaxClusterSplits;
+      if (cs < 1) cs = 1;
+    }
     long long cper = (window + cs - 1) / cs;
     cper = (cper + 15) / 16 * 16;
     s.slots_per_split = (int)cper;
     s.n_splits = (int)((window + cper - 1) / cper);
-    s.warps = warps;
+    s.warps = 8;
     s.cluster = s.n_splits > 1 ? 1 : 0;
+    s.stream = 1;
   }
   return s;
 }
@@ -331,6 +341,7 @@ const char* swa_last_error(void) { return g_last_error; }
 
 int swa_cache_append(const swa_dims* dims, void* k_cache, void* v_cache, const void* k, const void* v,
                      int32_t max_tokens, const int32_t* start_pos, const int32_t* n_tokens, void* stream) {
+  CallRange range_("swa_cache_append");
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_ptrs("k_cache, v_cache, k, v", {k_cache, v_cache, k, v}))) return rc;
@@ -367,6 +378,7 @@ size_t swa_prefill_workspace_size(const swa_dims* dims, int32_t max_tokens) {
 int swa_prefill_chunk(const swa_dims* dims, void* out, const void* q, const void* k, const void* v,
                       int32_t max_tokens, const void* k_cache, const void* v_cache, const int32_t* start_pos,
                       const int32_t* n_tokens, void* workspace, size_t workspace_bytes, void* stream) {
+  CallRange range_("swa_prefill_chunk");
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_ptrs("out, q, k, v, k_cache, v_cache", {out, q, k, v, k_cache, v_cache}))) return rc;
@@ -449,6 +461,7 @@ int swa_decode_launch_info(const swa_dims* dims, int32_t* n_splits, int32_t* n_l
 int swa_decode(const swa_dims* dims, void* out, const void* q, const void* k_new, const void* v_new,
                void* k_cache, void* v_cache, const int32_t* pos, void* workspace, size_t workspace_bytes,
                void* stream) {
+  CallRange range_("swa_decode");
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_ptrs("out, q, k_new, v_new, k_cache, v_cache, workspace",
@@ -485,6 +498,7 @@ int swa_decode(const swa_dims* dims, void* out, const void* q, const void* k_new
   p.slots_per_split = sp.slots_per_split;
   p.warps = sp.warps;
   p.cluster = sp.cluster;
+  p.stream = sp.stream;
   p.scale_log2 = dims->scale * 1.4426950408889634f;
   p.out_f32 = dims->out_dtype == SWA_DTYPE_F32;
   cudaError_t e = swa::launch_decode(p, static_cast<cudaStream_t>(stream));
@@ -493,6 +507,7 @@ int swa_decode(const swa_dims* dims, void* out, const void* q, const void* k_new
 }
 
 int swa_device_status(void* stream) {
+  CallRange range_("swa_device_status");
   int* status = nullptr;
   int rc = status_ptr(&status);
   if (rc) return rc;

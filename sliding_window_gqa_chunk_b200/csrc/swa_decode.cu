@@ -38,6 +38,7 @@
 
 #include "swa_common.cuh"
 #include "swa_internal.h"
+#include "swa_tc.cuh"
 
 namespace swa {
 
@@ -113,6 +114,80 @@ __device__ __forceinline__ void load_v_row(uint32_t (&w)[Frag<D>::kVWords], cons
   }
 }
 
+// Stream variant: the slots come from a shared-memory ring filled by bulk
+// copies.  Same fragments as load_k_row / load_v_row, read from the row at
+// shared address `srow`, or from global memory `grow` for the slot the new
+// key / value goes to (that slot's cache row is being rewritten).
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(a));
+  return r;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 r;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(a));
+  return r;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t r;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(a));
+  return r;
+}
+
+template <int D>
+__device__ __forceinline__ void load_k_row_s(uint32_t (&w)[Frag<D>::kKWords], uint32_t srow,
+                                             const __nv_bfloat16* grow, bool from_global, int t,
+                                             bool valid) {
+  if (!valid || from_global) {
+    load_k_row<D>(w, grow, t, valid);
+    return;
+  }
+  if constexpr (D == 16) {
+    uint2 x = lds64(srow + 2 * k_piece_offset<D>(t, 0));
+    w[0] = x.x;
+    w[1] = x.y;
+  } else {
+#pragma unroll
+    for (int j = 0; j < D / 32; ++j) {
+      uint4 x = lds128(srow + 2 * k_piece_offset<D>(t, j));
+      w[4 * j + 0] = x.x;
+      w[4 * j + 1] = x.y;
+      w[4 * j + 2] = x.z;
+      w[4 * j + 3] = x.w;
+    }
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void load_v_row_s(uint32_t (&w)[Frag<D>::kVWords], uint32_t srow,
+                                             const __nv_bfloat16* grow, bool from_global, int g,
+                                             bool valid) {
+  if (!valid || from_global) {
+    load_v_row<D>(w, grow, g, valid);
+    return;
+  }
+  if constexpr (D == 16) {
+    w[0] = lds32(srow + 2 * v_piece_offset<D>(g, 0));
+  } else {
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      uint4 x = lds128(srow + 2 * v_piece_offset<D>(g, c));
+      w[4 * c + 0] = x.x;
+      w[4 * c + 1] = x.y;
+      w[4 * c + 2] = x.z;
+      w[4 * c + 3] = x.w;
+    }
+  }
+}
+
+// Stream variant geometry: chunks of kChunkSlots slots (K rows and V rows,
+// each one contiguous range of the cache) in a ring of kStreamStages.
+constexpr int kChunkSlots = 64;
+constexpr int kStreamStages = 6;
+
+template <int D>
+constexpr int stream_ring_bytes() { return kStreamStages * 2 * kChunkSlots * D * 2; }
+
 // Programmatic dependent launch: the kernels below are launched with
 // programmatic stream serialization, so they may be scheduled while the
 // previous kernel in the stream is still running; this wait (first thing in
@@ -132,12 +207,15 @@ __device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* dst, flo
 
 }  // namespace
 
-// NT = number of 8-head n-tiles (ceil(G / 8)).
-template <int D, int NT, int NW, typename OutT>
-__global__ void __launch_bounds__(NW * 32)
+// NT = number of 8-head n-tiles (ceil(G / 8)); NW = compute warps.  STREAM:
+// one more warp streams the CTA's slots into a shared-memory ring with bulk
+// copies (every byte of the split in flight from the start), and the compute
+// warps read their fragments from there.
+template <int D, int NT, int NW, typename OutT, bool STREAM>
+__global__ void __launch_bounds__((NW + (STREAM ? 1 : 0)) * 32)
 swa_decode_kernel(const DecodeParams p) {
   using F = Frag<D>;
-  extern __shared__ float smem[];
+  extern __shared__ __align__(128) float smem[];
 
   const int split = blockIdx.x;
   const int kvh = blockIdx.y;
@@ -178,6 +256,54 @@ swa_decode_kernel(const DecodeParams p) {
     }
   }
 
+  // ---- stream variant: ring of K / V chunks, full / empty barriers ----
+  constexpr int G8 = 8 * NT;
+  constexpr int kMergeBytes = (int)sizeof(float) * (NW + 1) * G8 * (2 + D);
+  constexpr int kRingBytes = STREAM ? stream_ring_bytes<D>() : 0;
+  constexpr int kBarOffset = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
+  const uint32_t s_base = tc::smem_u32(smem);
+  const uint32_t sK = s_base;
+  const uint32_t sV = s_base + kStreamStages * kChunkSlots * D * 2;
+  const uint32_t bar_full = s_base + kBarOffset;          // [kStreamStages]
+  const uint32_t bar_empty = bar_full + 8 * kStreamStages;  // [kStreamStages]
+  bool stream_ok = true;
+  if constexpr (STREAM) {
+    if (threadIdx.x == 0) {
+      for (int i = 0; i < kStreamStages; ++i) {
+        tc::mbar_init(bar_full + 8 * i, 1);
+        tc::mbar_init(bar_empty + 8 * i, kChunkSlots / kBlockSlots);  // one arrival per block
+      }
+      tc::mbar_fence_init();
+    }
+    __syncthreads();
+    if (warp == NW) {
+      // Producer: chunk k of the split goes to stage k mod kStreamStages once
+      // the blocks of chunk k - kStreamStages have been read.
+      if (lane == 0) {
+        const int n_slots = r_end > r_begin ? r_end - r_begin : 0;
+        const int n_chunks = (n_slots + kChunkSlots - 1) / kChunkSlots;
+        int k = 0;
+        for (; k < n_chunks; ++k) {
+          const int st = k % kStreamStages;
+          if (k >= kStreamStages &&
+              !tc::mbar_wait(bar_empty + 8 * st, ((k / kStreamStages) - 1) & 1, p.status)) {
+            stream_ok = false;
+            break;
+          }
+          const int x = r_begin + k * kChunkSlots;
+          const int cnt = (r_end - x) < kChunkSlots ? (r_end - x) : kChunkSlots;
+          const uint32_t bytes = (uint32_t)cnt * D * 2;
+          tc::mbar_arrive_expect_tx(bar_full + 8 * st, 2 * bytes);
+          tc::bulk_load(sK + st * kChunkSlots * D * 2, kc + (size_t)x * D, bytes, bar_full + 8 * st);
+          tc::bulk_load(sV + st * kChunkSlots * D * 2, vc + (size_t)x * D, bytes, bar_full + 8 * st);
+        }
+        // every copy issued here has landed before the ring is reused
+        for (int j = k > kStreamStages ? k - kStreamStages : 0; j < k; ++j)
+          tc::mbar_wait(bar_full + 8 * (j % kStreamStages), (j / kStreamStages) & 1, p.status);
+      }
+    }
+  }
+
   // Q as the B operand of S^T = K Q^T: lane (g, t) holds head 8*nt + g.
   uint32_t qf[NT][F::kKWords];
 #pragma unroll
@@ -202,19 +328,40 @@ swa_decode_kernel(const DecodeParams p) {
   }
   const float sl2 = p.scale_log2;
 
-  for (int blk = r_begin + warp * kBlockSlots; blk < r_end; blk += NW * kBlockSlots) {
+  const int loop_end = (STREAM && warp >= NW) ? r_begin : r_end;  // the producer warp computes nothing
+  for (int blk = r_begin + warp * kBlockSlots; blk < loop_end; blk += NW * kBlockSlots) {
     // ---- loads: K rows blk+g, blk+8+g; V rows blk+2t, +1, +8, +9 ----
     uint32_t kw0[F::kKWords], kw1[F::kKWords];
-    {
+    uint32_t vw[4][F::kVWords];
+    if constexpr (STREAM) {
+      const int k = (blk - r_begin) / kChunkSlots;
+      const int st = k % kStreamStages;
+      stream_ok = __all_sync(0xffffffffu,
+                             tc::mbar_wait(bar_full + 8 * st, (k / kStreamStages) & 1, p.status));
+      if (!stream_ok) break;
+      const int in0 = blk - r_begin - k * kChunkSlots;  // first row of the block within the chunk
+      const uint32_t ks = sK + st * kChunkSlots * D * 2 + in0 * D * 2;
+      const uint32_t vs = sV + st * kChunkSlots * D * 2 + in0 * D * 2;
+      const int r0 = blk + g, r1 = blk + 8 + g;
+      load_k_row_s<D>(kw0, ks + g * D * 2, kn, r0 == s_new, t, r0 < r_end);
+      load_k_row_s<D>(kw1, ks + (8 + g) * D * 2, kn, r1 == s_new, t, r1 < r_end);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int ri = 2 * t + (i & 1) + (i >> 1) * 8;
+        const int r = blk + ri;
+        load_v_row_s<D>(vw[i], vs + ri * D * 2, vn, r == s_new, g, r < r_end);
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar_empty + 8 * st);  // this block's rows are in registers
+    } else {
       const int r0 = blk + g, r1 = blk + 8 + g;
       load_k_row<D>(kw0, r0 == s_new ? kn : kc + (size_t)r0 * D, t, r0 < r_end);
       load_k_row<D>(kw1, r1 == s_new ? kn : kc + (size_t)r1 * D, t, r1 < r_end);
-    }
-    uint32_t vw[4][F::kVWords];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = blk + 2 * t + (i & 1) + (i >> 1) * 8;
-      load_v_row<D>(vw[i], r == s_new ? vn : vc + (size_t)r * D, g, r < r_end);
+      for (int i = 0; i < 4; ++i) {
+        const int r = blk + 2 * t + (i & 1) + (i >> 1) * 8;
+        load_v_row<D>(vw[i], r == s_new ? vn : vc + (size_t)r * D, g, r < r_end);
+      }
     }
     const bool ok0 = blk + g < r_end;
     const bool ok1 = blk + 8 + g < r_end;
@@ -283,8 +430,12 @@ swa_decode_kernel(const DecodeParams p) {
 
   // ---- merge the NW warps of the CTA ----
   // smem: m[NW][G8], l[NW][G8], O[NW][G8][D] with G8 = 8*NT, then the CTA's
-  // partial m[G8], l[G8], O[G8][D] (cluster merge)
-  constexpr int G8 = 8 * NT;
+  // partial m[G8], l[G8], O[G8][D] (cluster merge); in the stream variant this
+  // reuses the ring, once every warp is done with it.
+  if constexpr (STREAM) {
+    if (!stream_ok && lane == 0) raise_status(p.status, SWA_ERR_TIMEOUT);
+    __syncthreads();
+  }
   float* sm_m = smem;
   float* sm_l = sm_m + NW * G8;
   float* sm_o = sm_l + NW * G8;
@@ -292,7 +443,7 @@ swa_decode_kernel(const DecodeParams p) {
   float* cta_l = cta_m + G8;
   float* cta_o = cta_l + G8;
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
+  for (int nt = 0; nt < NT && warp < NW; ++nt) {
     float l0 = l_run[nt][0], l1 = l_run[nt][1];
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
@@ -369,19 +520,35 @@ swa_decode_kernel(const DecodeParams p) {
     cl.sync();
     const int rank = (int)cl.block_rank();
     const int R = p.n_splits;
-    for (int idx = rank * blockDim.x + threadIdx.x; idx < G * D; idx += R * blockDim.x) {
+    // Rank r merges outputs [r * per, (r + 1) * per) of the G x d outputs, so
+    // every CTA takes an equal share; each thread fetches all R partials of
+    // its output with independent remote loads before combining them.
+    const int per = (G * D + R - 1) / R;
+    for (int idx = rank * per + threadIdx.x; idx < (rank + 1) * per && idx < G * D; idx += blockDim.x) {
       const int h = idx / D;
       const int dd = idx - h * D;
+      float m_r[kDecodeMaxClusterSplits], l_r[kDecodeMaxClusterSplits], o_r[kDecodeMaxClusterSplits];
+#pragma unroll
+      for (int r = 0; r < kDecodeMaxClusterSplits; ++r) {
+        if (r < R) {
+          m_r[r] = cl.map_shared_rank(cta_m, r)[h];
+          l_r[r] = cl.map_shared_rank(cta_l, r)[h];
+          o_r[r] = cl.map_shared_rank(cta_o, r)[h * D + dd];
+        } else {
+          m_r[r] = -CUDART_INF_F;
+          l_r[r] = o_r[r] = 0.f;
+        }
+      }
       float M = -CUDART_INF_F;
-      for (int r = 0; r < R; ++r) M = fmaxf(M, cl.map_shared_rank(cta_m, r)[h]);
+#pragma unroll
+      for (int r = 0; r < kDecodeMaxClusterSplits; ++r) M = fmaxf(M, m_r[r]);
       float L = 0.f, O = 0.f;
       if (M != -CUDART_INF_F) {
-        for (int r = 0; r < R; ++r) {
-          const float m = cl.map_shared_rank(cta_m, r)[h];
-          if (m == -CUDART_INF_F) continue;
-          const float sc = fast_exp2(m - M);
-          L += sc * cl.map_shared_rank(cta_l, r)[h];
-          O += sc * cl.map_shared_rank(cta_o, r)[h * D + dd];
+#pragma unroll
+        for (int r = 0; r < kDecodeMaxClusterSplits; ++r) {
+          const float sc = (m_r[r] == -CUDART_INF_F) ? 0.f : fast_exp2(m_r[r] - M);
+          L += sc * l_r[r];
+          O += sc * o_r[r];
         }
       }
       const size_t bh = (size_t)b * p.n_q_heads + hq0 + h;
@@ -417,14 +584,27 @@ swa_decode_combine_kernel(const DecodeParams p) {
 
 namespace {
 
-template <int D, int NT, int NW, typename OutT>
+constexpr int kMaxDevices = 64;
+
+template <int D, int NT, int NW, typename OutT, bool STREAM>
 cudaError_t launch_decode_t(const DecodeParams& p, cudaStream_t stream) {
   constexpr int G8 = 8 * NT;
-  const size_t smem = sizeof(float) * (size_t)(NW + 1) * G8 * (2 + D);
-  auto kern = swa_decode_kernel<D, NT, NW, OutT>;
+  constexpr size_t merge = sizeof(float) * (size_t)(NW + 1) * G8 * (2 + D);
+  constexpr size_t ring = STREAM ? (size_t)stream_ring_bytes<D>() : 0;
+  constexpr size_t smem = (ring > merge ? ring : merge) + (STREAM ? 16 * kStreamStages : 0);
+  auto kern = swa_decode_kernel<D, NT, NW, OutT, STREAM>;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // raised once per device (the attribute persists for the process)
+    static bool set[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (!set[dev]) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      set[dev] = true;
+    }
   }
   dim3 grid(p.n_splits, p.n_kv_heads, p.batch);
   cudaLaunchAttribute attr[2];
@@ -436,7 +616,7 @@ cudaError_t launch_decode_t(const DecodeParams& p, cudaStream_t stream) {
   attr[1].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(NW * 32);
+  cfg.blockDim = dim3((NW + (STREAM ? 1 : 0)) * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
@@ -455,12 +635,12 @@ cudaError_t launch_decode_t(const DecodeParams& p, cudaStream_t stream) {
 template <int D, typename OutT>
 cudaError_t launch_decode_d(const DecodeParams& p, cudaStream_t stream) {
   const int G = p.n_q_heads / p.n_kv_heads;
-  if (G <= 8) {
-    if (p.warps == 16) return launch_decode_t<D, 1, 16, OutT>(p, stream);
-    return launch_decode_t<D, 1, 4, OutT>(p, stream);
+  if (p.stream) {
+    if (G <= 8) return launch_decode_t<D, 1, 8, OutT, true>(p, stream);
+    return launch_decode_t<D, 2, 8, OutT, true>(p, stream);
   }
-  if (p.warps == 8) return launch_decode_t<D, 2, 8, OutT>(p, stream);
-  return launch_decode_t<D, 2, 4, OutT>(p, stream);
+  if (G <= 8) return launch_decode_t<D, 1, 4, OutT, false>(p, stream);
+  return launch_decode_t<D, 2, 4, OutT, false>(p, stream);
 }
 
 template <typename OutT>

@@ -31,6 +31,7 @@
 //     wrong results; order them on one stream or use swa_decode with separate
 //     workspaces.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <mutex>
 
@@ -43,6 +44,12 @@ constexpr size_t kStaticScratchBytes = 4u << 20;  // 4 MiB, same on every device
 
 // The decode's scratch for swa_decode_static: fp32 partials, 256-byte aligned.
 static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
+
+// NVTX range around the entry point (see swa_api.cu).
+struct StaticCallRange {
+  StaticCallRange() { nvtxRangePushA("swa_decode_static"); }
+  ~StaticCallRange() { nvtxRangePop(); }
+};
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
@@ -74,6 +81,7 @@ int scratch_address(void** out) {
 extern "C" SWA_API int swa_decode_static(const swa_dims* dims, void* out, const void* q, const void* k_new,
                                          const void* v_new, void* k_cache, void* v_cache, const int32_t* pos,
                                          void* stream) {
+  StaticCallRange range_;
   int rc = swa::api_check_decode(dims, out, q, k_new, v_new, k_cache, v_cache, pos);
   if (rc) return rc;
   // The scratch this launch really uses: none when one split covers the window
@@ -115,6 +123,7 @@ extern "C" SWA_API int swa_decode_static(const swa_dims* dims, void* out, const 
   p.slots_per_split = sp.slots_per_split;
   p.warps = sp.warps;
   p.cluster = sp.cluster;
+  p.stream = sp.stream;
   p.scale_log2 = dims->scale * 1.4426950408889634f;
   p.out_f32 = dims->out_dtype == SWA_DTYPE_F32;
   cudaError_t e = swa::launch_decode(p, static_cast<cudaStream_t>(stream));

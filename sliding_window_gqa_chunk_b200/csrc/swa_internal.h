@@ -39,9 +39,14 @@ struct DecodeParams {
   int cluster;                  // 1: the n_splits CTAs of a (sequence, kv head) form a
                                 // thread-block cluster and merge through distributed
                                 // shared memory (no workspace, no combine kernel)
+  int stream;                   // 1: a producer warp streams the slots into shared
+                                // memory with bulk copies (few (sequence, kv head) pairs)
   float scale_log2;             // scale * log2(e)
   int out_f32;
 };
+
+// Largest thread-block cluster of decode split CTAs (the portable cluster size).
+constexpr int kDecodeMaxClusterSplits = 8;
 
 // Split of the W slots of one (sequence, kv head) across CTAs; depends only
 // on the shape so that the workspace size is a function of the dims.
@@ -50,6 +55,7 @@ struct DecodeSplit {
   int slots_per_split;
   int warps;
   int cluster;
+  int stream;
   int ws_splits;   // splits the workspace is sized for (fp32 partials per split)
 };
 DecodeSplit decode_split(int batch, int n_q_heads, int n_kv_heads, int window);

@@ -380,8 +380,15 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
       bool ok = true;
       for (int it = 0; ok; ++it) {
         int item = p.n_items;
-        if (it == 0) item = blockIdx.x;
-        else if (p.persistent) item = (int)gridDim.x + atomicAdd(ws_ctr, 1);
+        if (it == 0) {
+          item = blockIdx.x;
+        } else if (p.persistent) {
+          const int got = atomicAdd(ws_ctr, 1);
+          // A counter below zero means the workspace was not zero-filled:
+          // stop instead of walking an unbounded item range.
+          if (got < 0) raise_status(p.status, SWA_ERR_DEVICE_ARG);
+          else item = (int)gridDim.x + got;
+        }
         const int slot = it & 1;
         if (it >= 2) ok = tc::mbar_wait(bar_item_empty + 8 * slot, ((it >> 1) - 1) & 1, p.status);
         if (!ok) break;

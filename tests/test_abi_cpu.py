@@ -154,13 +154,16 @@ def test_python_binding_refuses_to_run_without_the_library(tmp_path, monkeypatch
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,W,expect", [
-    (1, 32, 8, 4096, (8, 1)),     # 8 pairs: one cluster of 8 CTAs per pair, merged in-kernel
+    (1, 32, 8, 4096, (8, 1)),     # 8 pairs: a cluster of 8 streaming CTAs per pair, merged in-kernel
     (4, 32, 8, 4096, (8, 1)),     # 32 pairs: still clustered
-    (16, 32, 8, 4096, (4, 2)),    # 128 pairs: floor(592 / 128) = 4 splits + combine
+    (16, 32, 8, 4096, (1, 1)),    # 128 pairs (< 148 SMs): one streaming CTA per pair
+    (24, 32, 8, 4096, (3, 2)),    # 192 pairs: floor(592 / 192) = 3 splits + combine
+    (32, 32, 8, 4096, (2, 2)),    # 256 pairs: 2 splits + combine
     (64, 32, 8, 4096, (1, 1)),    # 512 pairs: one split, no combine
     (128, 32, 8, 4096, (1, 1)),
-    (2, 8, 2, 300, (2, 1)),       # cluster of 2 CTAs (300 slots, 256 per 16-warp CTA sweep)
-    (3, 12, 4, 100, (1, 1)),      # one CTA covers the window
+    (2, 8, 2, 1000, (2, 1)),      # cluster of 2 CTAs (about 512 slots each)
+    (2, 8, 2, 300, (1, 1)),       # one CTA covers the window
+    (3, 12, 4, 100, (1, 1)),
 ])
 def test_decode_launch_info_follows_the_split_rule(B, Hq, Hkv, W, expect):
     d = swa.Dims(B, Hq, Hkv, 128, W, 0.1, "bf16")

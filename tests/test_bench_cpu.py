@@ -95,10 +95,12 @@ def test_profiled_traffic_is_dropped_when_the_kernel_changes(monkeypatch):
 def test_decode_launch_count_follows_the_split_rule():
     import sliding_window_gqa_chunk_b200 as swa
     mk = lambda B: swa.Dims(B, 32, 8, 128, 4096, 1.0 / 128 ** 0.5, "bf16")
-    # batch 1 and 4: one launch (clustered splits); 16: 4 splits + combine;
-    # 64 and 128: one split per (sequence, kv head), no combine
+    # batch 1 and 4: one launch (clustered splits); 16: one streaming CTA per
+    # (sequence, kv head); 24: 3 splits + combine; 64 and 128: one split per
+    # (sequence, kv head), no combine
     assert bench.decode_launches_per_call(mk(1), swa) == 1
     assert bench.decode_launches_per_call(mk(4), swa) == 1
-    assert bench.decode_launches_per_call(mk(16), swa) == 2
+    assert bench.decode_launches_per_call(mk(16), swa) == 1
+    assert bench.decode_launches_per_call(mk(24), swa) == 2
     assert bench.decode_launches_per_call(mk(64), swa) == 1
     assert bench.decode_launches_per_call(mk(128), swa) == 1

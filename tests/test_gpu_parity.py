@@ -74,7 +74,7 @@ def test_tiny_workload_prefill_then_decode(out_dtype):
         assert_close(o.double().cpu().numpy(), expect, f"chunk {c}", bf16_out=bf)
         np.testing.assert_array_equal(cache_as_f64(kc), ref.k)
         np.testing.assert_array_equal(cache_as_f64(vc), ref.v)
-    ws = torch.empty(swa.decode_workspace_size(dims), dtype=torch.uint8, device=DEV)
+    ws = swa.decode_workspace(dims, DEV)
     for i, (q, k, v) in enumerate(steps):
         p = 12 + i
         o = torch.zeros((1, s.n_q_heads, s.head_dim), dtype=dims.torch_out_dtype, device=DEV)
@@ -161,7 +161,7 @@ def test_prefill_chunk_after_decode_steps():
     dims = mk_dims(B, Hq, Hkv, d, W)
     kc, vc = swa.new_cache(dims, DEV)
     ref = oracle.RollingCache(B, Hkv, W, d)
-    ws = torch.empty(swa.decode_workspace_size(dims), dtype=torch.uint8, device=DEV)
+    ws = swa.decode_workspace(dims, DEV)
     for p in range(first):
         o = torch.zeros((B, Hq, d), dtype=torch.float32, device=DEV)
         swa.decode(dims, o, q[:, p].contiguous().to(DEV), k[:, p].contiguous().to(DEV),
@@ -193,6 +193,10 @@ DECODE_CASES = [
     (1, 16, 16, 1, 16, [3], 20),               # G = 16, wraps several times
     (5, 1000, 4, 4, 64, [0, 1, 2, 999, 1000], 2),  # G = 1
     (2, 4096, 64, 8, 128, [70000, 4095], 2),   # G = 8
+    # 80 pairs: one streaming CTA per pair, 11 chunks with a partial last one,
+    # caches from empty to wrapped
+    (10, 700, 16, 8, 64, [0, 5, 699, 700, 1500, 33, 2000, 64, 65, 128], 2),
+    (6, 2048, 32, 8, 128, [9000, 2047, 2048, 100, 3000, 4100], 2),  # 48 pairs: clusters of 4
 ]
 
 
@@ -212,7 +216,7 @@ def test_decode_matches_oracle(B, W, Hq, Hkv, d, pos0, steps):
             vc[b, :, p % W] = vr
             ref.write(b, p, kr, vr)
     kc, vc = kc.to(DEV), vc.to(DEV)
-    ws = torch.empty(swa.decode_workspace_size(dims), dtype=torch.uint8, device=DEV)
+    ws = swa.decode_workspace(dims, DEV)
     for s in range(steps):
         pos = [p + s for p in pos0]
         q = torch.randn(B, Hq, d, generator=g).to(torch.bfloat16)
@@ -242,7 +246,7 @@ def test_decode_bf16_output():
     k = torch.randn(B, Hkv, d, generator=g).to(torch.bfloat16)
     v = torch.randn(B, Hkv, d, generator=g).to(torch.bfloat16)
     kcd, vcd = kc.to(DEV), vc.to(DEV)
-    ws = torch.empty(swa.decode_workspace_size(dims), dtype=torch.uint8, device=DEV)
+    ws = swa.decode_workspace(dims, DEV)
     o = torch.zeros((B, Hq, d), dtype=torch.bfloat16, device=DEV)
     swa.decode(dims, o, q.to(DEV), k.to(DEV), v.to(DEV), kcd, vcd, dev_i32(pos), ws)
     expect = oracle.decode(ref, q, k, v, pos, dims.scale)

@@ -4,8 +4,9 @@ tensor pointers).  It takes no workspace; its scratch is an array built into
 the library.
 
 The dims here take the path that really uses that scratch: enough (sequence,
-kv head) pairs that the splits of the cache sweep are merged through memory
-by a second kernel (swa_decode_launch_info reports two launches).  Two calls
+kv head) pairs (more than the SMs) that the splits of the cache sweep are
+merged through memory by a second kernel (swa_decode_launch_info reports two
+launches).  Two calls
 in a row are checked against swa_decode with a caller workspace and against
 the float64 oracle; then calls with other dims (another split count and batch,
 so another partial layout over the same scratch) show that nothing stale from
@@ -66,16 +67,16 @@ def _run_case(B, W, Hq, Hkv, d, expect_splits, seed):
 
 
 def test_static_decode_uses_its_scratch_and_matches_on_two_calls():
-    # 16 x 8 = 128 (sequence, kv head) pairs: 4 splits of 1024 slots each,
-    # merged by the combine kernel through 1.06 MB of the built-in scratch
-    _run_case(B=16, W=4096, Hq=32, Hkv=8, d=128, expect_splits=4, seed=123)
+    # 24 x 8 = 192 (sequence, kv head) pairs: 3 splits of 1408 slots each,
+    # merged by the combine kernel through 1.2 MB of the built-in scratch
+    _run_case(B=24, W=4096, Hq=32, Hkv=8, d=128, expect_splits=3, seed=123)
 
 
 def test_static_decode_after_other_dims_sees_no_stale_scratch():
-    # run after the case above: 64 pairs, 8 splits of 128 slots, another layout
-    # of partials over the same scratch bytes
-    _run_case(B=8, W=1024, Hq=32, Hkv=8, d=128, expect_splits=8, seed=7)
-    _run_case(B=16, W=4096, Hq=32, Hkv=8, d=128, expect_splits=4, seed=8)
+    # run after the case above: 256 pairs, 2 splits, another layout of partials
+    # over the same scratch bytes, then the first dims again
+    _run_case(B=32, W=4096, Hq=32, Hkv=8, d=128, expect_splits=2, seed=7)
+    _run_case(B=24, W=4096, Hq=32, Hkv=8, d=128, expect_splits=3, seed=8)
 
 
 def test_static_decode_refuses_dims_beyond_its_scratch():
