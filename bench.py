@@ -688,9 +688,15 @@ def oracle_rows(wl, seed: int = 0):
     return torch.randperm(wl.lengths[0], generator=g).tolist()
 
 
+def oracle_inputs(wl):
+    """The workload's q/k/v widened once to float64 numpy (outside any timing)."""
+    q, k, v = prefill_inputs(wl, device="cpu")
+    return tuple(x.double().numpy() for x in (q, k, v))
+
+
 def oracle_sample(wl, rows, q, k, v):
     """The oracle on the given query rows (all heads, each row against its
-    window of keys from the full history): returns seconds."""
+    window of keys from the full history; float64 inputs): returns seconds."""
     import numpy as np
     import oracle
     W = wl.shape.window
@@ -710,7 +716,7 @@ def sample_note(n_rows, wl):
 
 def cpu_baseline(wl, budget_s=12.0):
     import oracle
-    q, k, v = prefill_inputs(wl, device="cpu")
+    q, k, v = oracle_inputs(wl)
     order = oracle_rows(wl)
     done, spent, batch = 0, 0.0, 32
     while spent < budget_s and done + batch <= len(order):
@@ -726,7 +732,7 @@ def bench_reference(args, world, rank):
     import oracle
     oracle.build()
     wl = PREFILL_16K
-    q, k, v = prefill_inputs(wl, device="cpu")
+    q, k, v = oracle_inputs(wl)
     rows = args.ref_rows
     order = oracle_rows(wl, seed=1)
     for i in range(args.warmup):

@@ -196,6 +196,14 @@ constexpr int stream_ring_bytes() { return kStreamStages * 2 * kChunkSlots * D *
 // write.  Only the launch latency is overlapped.
 __device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Lets the next kernel in the stream (launched with programmatic stream
+// serialization) be scheduled onto free SMs now instead of at this kernel's
+// end; it still waits in wait_prior_grid for this kernel to complete.  Issued
+// right after this kernel's own wait, so at most one kernel runs ahead.
+__device__ __forceinline__ void allow_next_grid() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 template <typename OutT>
 __device__ __forceinline__ void store_out(OutT* dst, float x);
 template <>
@@ -228,6 +236,7 @@ swa_decode_kernel(const DecodeParams p) {
   const int W = p.window;
 
   wait_prior_grid();
+  allow_next_grid();
   const long long pos = p.pos[b];
   if (pos < 0) {
     if (threadIdx.x == 0) raise_status(p.status, SWA_ERR_DEVICE_ARG);
@@ -563,6 +572,7 @@ template <int D, typename OutT>
 __global__ void __launch_bounds__(D < 32 ? 32 : D)
 swa_decode_combine_kernel(const DecodeParams p) {
   wait_prior_grid();
+  allow_next_grid();
   const size_t bh = blockIdx.x;
   const int dd = threadIdx.x;
   if (dd >= D) return;

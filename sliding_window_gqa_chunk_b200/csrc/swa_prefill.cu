@@ -9,7 +9,8 @@
 //   warp  8    TMA producer: Q once, then K tiles into an NK-stage ring
 //   warp  9    TMEM allocator and MMA issuer (one elected lane issues tcgen05.mma)
 //   warp 10    TMA producer: V tiles into an NV-stage ring
-//   warp 11    idle (it completes the third warpgroup)
+//   warp 11    work fetcher: takes units (or pieces of units) and publishes
+//              them to the other roles through a two-entry ring
 // The kernel is compiled for 168 registers per thread (12 warps); the third
 // warpgroup gives registers back (setmaxnreg) so that each softmax thread can
 // hold its whole 128-column row of S without spilling.
@@ -68,12 +69,13 @@ constexpr int kThreads = 384;       // 12 warps = 3 warpgroups
 // block's register pool), or setmaxnreg.inc would wait forever; the host
 // refuses to launch if ptxas did not allocate exactly kLaunchRegs.
 constexpr int kLaunchRegs = 168;
-constexpr int kSoftmaxRegs = 208;
-constexpr int kOtherRegs = 88;
+constexpr int kSoftmaxRegs = 224;
+constexpr int kOtherRegs = 56;
 static_assert(2 * kSoftmaxRegs + kOtherRegs == 3 * kLaunchRegs, "register split must fill the pool");
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kVProducerWarp = 10;
+constexpr int kFetchWarp = 11;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
 constexpr uint32_t kTmemCols = 512;
 // Workspace layout: two scheduler counters; one merge counter per split unit
@@ -93,6 +95,11 @@ static_assert(kWsMergeOffset + kMaxPersistentCtas * 8 * sizeof(int) <= kWsPartia
 #define SWA_EXP2_FMA_PAIRS 0x00
 #endif
 
+// 1: the two heads' softmax warps of a sub-partition alternate their
+// exponential passes (see the softmax loop); 0: they run unsynchronised.
+#ifndef SWA_SOFTMAX_PINGPONG
+#define SWA_SOFTMAX_PINGPONG 1
+#endif
 // K / V ring depths for head_dim 128 (2 Q tiles + K + V must fit in 227 KB).
 #ifndef SWA_K_STAGES_D128
 #define SWA_K_STAGES_D128 3
@@ -153,8 +160,11 @@ __device__ __forceinline__ TilePlan make_plan(long long s, int t_lo, int qt, int
     pl.first_cache = 0;
     return pl;
   }
-  const int a = (int)(c_lo % W);
-  const int last = (int)((c_lo + n_c - 1) % W);
+  // Positions are below 2^32 (start_pos is an int32 and t < W), so the
+  // slot arithmetic runs in 32-bit unsigned (a 64-bit remainder is a long
+  // subroutine that would cost the producer warps registers).
+  const int a = (int)((uint32_t)c_lo % (uint32_t)W);
+  const int last = (int)((uint32_t)(c_lo + n_c - 1) % (uint32_t)W);
   const int ft = a / kKeys, lt = last / kKeys;
   if (a + n_c <= W) {
     pl.first_cache = ft;
@@ -277,6 +287,61 @@ __device__ __forceinline__ float ld_cg(const float* a) {
   return v;
 }
 
+// An item as the fetcher warp publishes it in shared memory: the fields every
+// role needs, so that no other role repeats the decoding (its divisions and
+// global loads would sit on the critical path of each item and cost
+// registers in the producer warpgroup).
+constexpr int kRecInts = 20;
+enum RecField {
+  kRecEnd = 0, kRecB, kRecKvh, kRecHFirst, kRecTLo, kRecS, kRecN, kRecPiece, kRecNp, kRecMerge,
+  kRecSlot, kRecJ0, kRecNTiles, kRecNCache, kRecFirstCache, kRecNWTiles, kRecNChunk
+};
+
+__device__ __forceinline__ void rec_store(volatile int* r, const Item& I, bool end) {
+  r[kRecEnd] = end ? 1 : 0;
+  if (end) return;
+  r[kRecB] = I.b;
+  r[kRecKvh] = I.kvh;
+  r[kRecHFirst] = I.h_first;
+  r[kRecTLo] = I.t_lo;
+  r[kRecS] = (int)I.s;
+  r[kRecN] = I.n;
+  r[kRecPiece] = I.piece;
+  r[kRecNp] = I.np;
+  r[kRecMerge] = I.merge_idx;
+  r[kRecSlot] = I.slot;
+  r[kRecJ0] = I.j0;
+  r[kRecNTiles] = I.n_tiles;
+  r[kRecNCache] = I.plan.n_cache;
+  r[kRecFirstCache] = I.plan.first_cache;
+  r[kRecNWTiles] = I.plan.n_wtiles;
+  r[kRecNChunk] = I.plan.n_chunk;
+}
+
+__device__ __forceinline__ Item rec_load(const volatile int* r) {
+  Item I;
+  I.b = r[kRecB];
+  I.kvh = r[kRecKvh];
+  I.h_first = r[kRecHFirst];
+  I.t_lo = r[kRecTLo];
+  I.qt = I.t_lo / kRows;
+  I.s = r[kRecS];
+  I.n = r[kRecN];
+  I.rows = true;
+  I.bad_args = false;
+  I.piece = r[kRecPiece];
+  I.np = r[kRecNp];
+  I.merge_idx = r[kRecMerge];
+  I.slot = r[kRecSlot];
+  I.j0 = r[kRecJ0];
+  I.n_tiles = r[kRecNTiles];
+  I.plan.n_cache = r[kRecNCache];
+  I.plan.first_cache = r[kRecFirstCache];
+  I.plan.n_wtiles = r[kRecNWTiles];
+  I.plan.n_chunk = r[kRecNChunk];
+  return I;
+}
+
 }  // namespace
 
 template <int D, typename OutT>
@@ -314,12 +379,14 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
   const uint32_t bar_item_full = bar_o_full + 16;      // [2]
   const uint32_t bar_item_empty = bar_item_full + 16;  // [2]
   const uint32_t bar_done = bar_item_empty + 16;
-  static_assert(16 + 16 * NK + 16 * NV + 6 * 16 + 8 <= 256, "barrier area");
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::kSmemTiles + 256);
-  volatile int* item_q = reinterpret_cast<volatile int*>(base_ptr + C::kSmemTiles + 264);  // [2]
-  // Consumers of the item queue: the V producer, the MMA warp and every
-  // softmax warp (one arrival each).
-  const int n_item_consumers = 2 + 4 * hpc;
+  const uint32_t bar_turn = bar_done + 8;              // [2 heads][4 sub-partitions]
+  static_assert(16 + 16 * NK + 16 * NV + 5 * 16 + 8 + 64 <= 320, "barrier area");
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::kSmemTiles + 320);
+  volatile int* item_rec = reinterpret_cast<volatile int*>(base_ptr + C::kSmemTiles + 336);  // [2][kRecInts]
+  static_assert(336 + 2 * kRecInts * 4 <= 512, "item records must fit the control area");
+  // Consumers of the item queue: the K and V producers, the MMA warp and
+  // every softmax warp (one arrival each).
+  const int n_item_consumers = 3 + 4 * hpc;
 
   if (threadIdx.x == 0) {
     tc::mbar_init(bar_q_full, 1);
@@ -340,6 +407,7 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
       tc::mbar_init(bar_item_empty + 8 * i, n_item_consumers);
     }
     tc::mbar_init(bar_done, 1);
+    for (int i = 0; i < 8; ++i) tc::mbar_init(bar_turn + 8 * i, 1);
     tc::mbar_fence_init();
   }
   if (threadIdx.x == 0) SWA_TRACE_AT(0, 1);
@@ -354,33 +422,30 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) SWA_TRACE_AT(0, 3);
 
-  // Item queue: the K producer fetches items (the CTA's own index first, then
-  // from the shared counter when the grid is persistent) and publishes each in
-  // a two-entry ring; every other role reads the same sequence.  An index
-  // >= n_items ends the sequence.
-  auto next_item = [&](int it, bool& ok) -> int {
+  // Item queue: the fetcher warp takes items (the CTA's own index first, then
+  // from the shared counter when the grid is persistent), skips units with no
+  // query rows, and publishes each remaining item as a record in a two-entry
+  // ring; every other role reads the same sequence.  A record with the end
+  // flag closes it.  Consumers read the fields they need before they release
+  // the entry.
+  auto wait_item = [&](int it, bool& ok) -> const volatile int* {
     const int slot = it & 1;
     ok = tc::mbar_wait(bar_item_full + 8 * slot, (it >> 1) & 1, p.status);
-    const int item = ok ? item_q[slot] : p.n_items;
-    return item;
+    return item_rec + slot * kRecInts;
   };
 
   // setmaxnreg is per warpgroup and must dominate the code it budgets, so the
   // role dispatch happens inside the two register branches.
   if (warp >= 8) {
   tc::regs_decrease<kOtherRegs>();
-  if (warp == kProducerWarp) {
-    // =============== item fetcher and TMA producer: Q, then K tiles ===============
+  if (warp == kFetchWarp) {
+    // ================================ item fetcher ================================
     if (lane == 0) {
-      tc::prefetch_map(&maps.q);
-      tc::prefetch_map(&maps.k);
-      tc::prefetch_map(&maps.kc);
-      int kt = 0;   // K tiles issued (ring position)
-      int qi = 0;   // Q tiles issued (items with tiles)
       bool ok = true;
-      for (int it = 0; ok; ++it) {
+      int pub = 0;  // records published
+      for (int fetch = 0; ok; ++fetch) {
         int item = p.n_items;
-        if (it == 0) {
+        if (fetch == 0) {
           item = blockIdx.x;
         } else if (p.persistent) {
           const int got = atomicAdd(ws_ctr, 1);
@@ -389,16 +454,41 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
           if (got < 0) raise_status(p.status, SWA_ERR_DEVICE_ARG);
           else item = (int)gridDim.x + got;
         }
-        const int slot = it & 1;
-        if (it >= 2) ok = tc::mbar_wait(bar_item_empty + 8 * slot, ((it >> 1) - 1) & 1, p.status);
-        if (!ok) break;
         if (item > p.n_items) item = p.n_items;
-        item_q[slot] = item;
+        const bool end = item >= p.n_items;
+        Item I;
+        if (!end) {
+          I = decode_item(p, item);
+          if (I.bad_args && I.qt == 0 && I.piece == 0 && I.h_first == 0)
+            raise_status(p.status, SWA_ERR_DEVICE_ARG);
+          if (!I.rows) continue;  // no query rows: nothing for the other roles
+        }
+        const int slot = pub & 1;
+        if (pub >= 2) ok = tc::mbar_wait(bar_item_empty + 8 * slot, ((pub >> 1) - 1) & 1, p.status);
+        if (!ok) break;
+        rec_store(item_rec + slot * kRecInts, I, end);
         tc::mbar_arrive(bar_item_full + 8 * slot);
-        if (item >= p.n_items) break;
-        const Item I = decode_item(p, item);
-        if (I.bad_args && I.qt == 0 && I.piece == 0 && I.h_first == 0)
-          raise_status(p.status, SWA_ERR_DEVICE_ARG);
+        ++pub;
+        if (end) break;
+      }
+    }
+  } else if (warp == kProducerWarp) {
+    // ======================== TMA producer: Q, then K tiles ========================
+    if (lane == 0) {
+      tc::prefetch_map(&maps.q);
+      tc::prefetch_map(&maps.k);
+      tc::prefetch_map(&maps.kc);
+      int kt = 0;   // K tiles issued (ring position)
+      int qi = 0;   // Q tiles issued (items with tiles)
+      bool ok = true;
+      for (int it = 0; ok; ++it) {
+        const volatile int* rec = wait_item(it, ok);
+        if (!ok) break;
+        const bool end = rec[kRecEnd] != 0;
+        Item I;
+        if (!end) I = rec_load(rec);
+        tc::mbar_arrive(bar_item_empty + 8 * (it & 1));
+        if (end) break;
         if (I.n_tiles == 0) continue;
         SWA_TRACE_AT(1, 1000 + it);
         if (qi > 0) ok = tc::mbar_wait(bar_q_empty, (qi - 1) & 1, p.status);
@@ -449,10 +539,13 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
       int vt = 0;
       bool ok = true;
       for (int it = 0; ok; ++it) {
-        const int item = next_item(it, ok);
+        const volatile int* rec = wait_item(it, ok);
+        if (!ok) break;
+        const bool end = rec[kRecEnd] != 0;
+        Item I;
+        if (!end) I = rec_load(rec);
         tc::mbar_arrive(bar_item_empty + 8 * (it & 1));
-        if (!ok || item >= p.n_items) break;
-        const Item I = decode_item(p, item);
+        if (end) break;
         for (int j = 0; j < I.n_tiles; ++j, ++vt) {
           bool is_cache;
           int kbase;
@@ -518,17 +611,18 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
       int qi = 0;   // items with tiles
       bool ok = true;
       for (int it = 0; ok; ++it) {
-        int item;
+        const volatile int* rec;
         {
           bool got;
-          item = next_item(it, got);
+          rec = wait_item(it, got);
           ok = __all_sync(0xffffffffu, got);
         }
+        if (!ok) break;
+        const bool end = rec[kRecEnd] != 0;
+        const int n_tiles = end ? 0 : rec[kRecNTiles];
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(bar_item_empty + 8 * (it & 1));
-        if (!ok || item >= p.n_items) break;
-        const Item I = decode_item(p, item);
-        const int n_tiles = I.n_tiles;
+        if (end) break;
         if (n_tiles == 0) continue;
         ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_q_full, qi & 1, p.status));
         if (!ok) break;
@@ -597,17 +691,19 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
     int oi = 0;   // items with tiles (O barrier phase)
     bool ok = true;
     for (int it = 0; ok; ++it) {
-      int item;
+      const volatile int* rec;
       {
         bool got;
-        item = next_item(it, got);
+        rec = wait_item(it, got);
         ok = __all_sync(0xffffffffu, got);
       }
+      if (!ok) break;
+      const bool end = rec[kRecEnd] != 0;
+      Item I;
+      if (!end) I = rec_load(rec);
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(bar_item_empty + 8 * (it & 1));
-      if (!ok || item >= p.n_items) break;
-      const Item I = decode_item(p, item);
-      if (!I.rows) continue;
+      if (end) break;
       const int n_tiles = I.n_tiles;
       const int t = I.t_lo + row;               // chunk row
       const long long s = I.s;
@@ -616,7 +712,7 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
       long long lo_i = pos_i - W + 1;
       if (lo_i < 0) lo_i = 0;
       const int len_i = (int)(s - lo_i);          // <= W - 1; <= 0 means none
-      const int a_i = (int)(lo_i % W);
+      const int a_i = (int)((uint32_t)lo_i % (uint32_t)W);
 
       float m_run = -CUDART_INF_F;
       float l_run = 0.f;
@@ -717,6 +813,20 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
         // than 2^8 (always on a row's first visible tile) is the tile redone
         // against the new max.  The decisions are warp-uniform because the
         // TMEM accesses they guard are warp-collective.
+#if SWA_SOFTMAX_PINGPONG
+        // The two heads' softmax warps of one SM sub-partition share its SFU.
+        // They take turns on their exponential passes (head 0 of tile g, head
+        // 1 of tile g, head 0 of tile g + 1, ...) instead of running side by
+        // side at half speed each, so that one head's products run on the
+        // tensor core while the other head exponentiates.
+        if (hpc == 2) {
+          const int gt = g0 + j;
+          const uint32_t my_turn = bar_turn + 8 * (i * 4 + (warp & 3));
+          if (i == 1 || gt > 0)
+            ok = __all_sync(0xffffffffu, tc::mbar_wait(my_turn, (i == 0 ? gt - 1 : gt) & 1, p.status));
+          if (!ok) break;
+        }
+#endif
         float part = 0.f;
         bool exact = __any_sync(0xffffffffu, m_run == -CUDART_INF_F);
         if (!exact) {
@@ -766,6 +876,12 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
           part = exp_pass((m_run == -CUDART_INF_F) ? 0.f : -m_run, false, unused);
         }
         l_run += part;
+#if SWA_SOFTMAX_PINGPONG
+        if (hpc == 2) {  // hand the sub-partition's SFU to the other head
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(bar_turn + 8 * ((1 - i) * 4 + (warp & 3)));
+        }
+#endif
         tc::tc_wait_st();
         tc::tc_fence_before();
         __syncwarp();

@@ -39,8 +39,10 @@ def test_kv_head_shards_reassemble_to_the_oracle(Hq, Hkv, world):
             n = min(chunk, L - st)
             sp, nt = dev_i32([st] * B), dev_i32([n] * B)
             qc, kc_in, vc_in = (x[:, st:st + n].contiguous() for x in (qs, ks, vs))
-            swa.prefill_chunk(sd, out[:, st:st + n], qc, kc_in, vc_in, kc, vc, sp, nt, workspace=ws)
+            oc = torch.zeros((B, n, s.n_q_heads, d), dtype=torch.float32, device=DEV)
+            swa.prefill_chunk(sd, oc, qc, kc_in, vc_in, kc, vc, sp, nt, workspace=ws)
             swa.cache_append(sd, kc, vc, kc_in, vc_in, sp, nt)
+            out[:, st:st + n] = oc
         prefill_out.append(out.cpu())
         dws = swa.decode_workspace(sd, DEV)
         for i in range(steps):
