@@ -644,7 +644,7 @@ def bench_ours(args, world, rank, local):
 
     if phase in ("all", "decode32"):
         rows = []
-        for B in (1, 16, 64, 128):
+        for B in args.batches:
             dr = Decode32Run(decode_32l_workload(B), "bf16", dev)
             dr.capture()
             barrier(world)
@@ -769,6 +769,9 @@ def main(argv=None):
     ap.add_argument("--phase", choices=["all", "prefill", "decode", "dense", "varlen", "decode32"],
                     default="all",
                     help="run one phase only (for profiling); the headline line needs 'all'")
+    ap.add_argument("--batches", type=lambda x: [int(b) for b in x.split(",")],
+                    default=[1, 16, 64, 128],
+                    help="batch sizes of the 32-layer decode phase (comma list)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -69,8 +69,8 @@ constexpr int kThreads = 384;       // 12 warps = 3 warpgroups
 // block's register pool), or setmaxnreg.inc would wait forever; the host
 // refuses to launch if ptxas did not allocate exactly kLaunchRegs.
 constexpr int kLaunchRegs = 168;
-constexpr int kSoftmaxRegs = 224;
-constexpr int kOtherRegs = 56;
+constexpr int kSoftmaxRegs = 208;
+constexpr int kOtherRegs = 88;
 static_assert(2 * kSoftmaxRegs + kOtherRegs == 3 * kLaunchRegs, "register split must fill the pool");
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
@@ -95,11 +95,6 @@ static_assert(kWsMergeOffset + kMaxPersistentCtas * 8 * sizeof(int) <= kWsPartia
 #define SWA_EXP2_FMA_PAIRS 0x00
 #endif
 
-// 1: the two heads' softmax warps of a sub-partition alternate their
-// exponential passes (see the softmax loop); 0: they run unsynchronised.
-#ifndef SWA_SOFTMAX_PINGPONG
-#define SWA_SOFTMAX_PINGPONG 1
-#endif
 // K / V ring depths for head_dim 128 (2 Q tiles + K + V must fit in 227 KB).
 #ifndef SWA_K_STAGES_D128
 #define SWA_K_STAGES_D128 3
@@ -379,8 +374,8 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
   const uint32_t bar_item_full = bar_o_full + 16;      // [2]
   const uint32_t bar_item_empty = bar_item_full + 16;  // [2]
   const uint32_t bar_done = bar_item_empty + 16;
-  const uint32_t bar_turn = bar_done + 8;              // [2 heads][4 sub-partitions]
-  static_assert(16 + 16 * NK + 16 * NV + 5 * 16 + 8 + 64 <= 320, "barrier area");
+  const uint32_t bar_fetch = bar_done + 8;             // K producer done issuing an item
+  static_assert(16 + 16 * NK + 16 * NV + 5 * 16 + 16 <= 320, "barrier area");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::kSmemTiles + 320);
   volatile int* item_rec = reinterpret_cast<volatile int*>(base_ptr + C::kSmemTiles + 336);  // [2][kRecInts]
   static_assert(336 + 2 * kRecInts * 4 <= 512, "item records must fit the control area");
@@ -407,7 +402,7 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
       tc::mbar_init(bar_item_empty + 8 * i, n_item_consumers);
     }
     tc::mbar_init(bar_done, 1);
-    for (int i = 0; i < 8; ++i) tc::mbar_init(bar_turn + 8 * i, 1);
+    tc::mbar_init(bar_fetch, 1);
     tc::mbar_fence_init();
   }
   if (threadIdx.x == 0) SWA_TRACE_AT(0, 1);
@@ -445,6 +440,14 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
       int pub = 0;  // records published
       for (int fetch = 0; ok; ++fetch) {
         int item = p.n_items;
+        // Take the next unit only once the K producer has issued the last
+        // tile of the previous one (a few tiles before the CTA finishes it),
+        // so that units go to CTAs close to the moment they can start them:
+        // greedy longest-first over the SMs, not a round-robin two units deep.
+        if (pub > 0 && fetch > 0) {
+          ok = tc::mbar_wait(bar_fetch, (pub - 1) & 1, p.status);
+          if (!ok) break;
+        }
         if (fetch == 0) {
           item = blockIdx.x;
         } else if (p.persistent) {
@@ -489,7 +492,10 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
         if (!end) I = rec_load(rec);
         tc::mbar_arrive(bar_item_empty + 8 * (it & 1));
         if (end) break;
-        if (I.n_tiles == 0) continue;
+        if (I.n_tiles == 0) {
+          tc::mbar_arrive(bar_fetch);
+          continue;
+        }
         SWA_TRACE_AT(1, 1000 + it);
         if (qi > 0) ok = tc::mbar_wait(bar_q_empty, (qi - 1) & 1, p.status);
         if (!ok) break;
@@ -520,6 +526,7 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
                               bar_k_full + 8 * sk);
           }
         }
+        if (ok) tc::mbar_arrive(bar_fetch);  // the fetcher may take the next unit now
       }
       // Before leaving, make sure no copy issued here is still in flight: the
       // last Q load and the last use of every K stage.
@@ -813,20 +820,6 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
         // than 2^8 (always on a row's first visible tile) is the tile redone
         // against the new max.  The decisions are warp-uniform because the
         // TMEM accesses they guard are warp-collective.
-#if SWA_SOFTMAX_PINGPONG
-        // The two heads' softmax warps of one SM sub-partition share its SFU.
-        // They take turns on their exponential passes (head 0 of tile g, head
-        // 1 of tile g, head 0 of tile g + 1, ...) instead of running side by
-        // side at half speed each, so that one head's products run on the
-        // tensor core while the other head exponentiates.
-        if (hpc == 2) {
-          const int gt = g0 + j;
-          const uint32_t my_turn = bar_turn + 8 * (i * 4 + (warp & 3));
-          if (i == 1 || gt > 0)
-            ok = __all_sync(0xffffffffu, tc::mbar_wait(my_turn, (i == 0 ? gt - 1 : gt) & 1, p.status));
-          if (!ok) break;
-        }
-#endif
         float part = 0.f;
         bool exact = __any_sync(0xffffffffu, m_run == -CUDART_INF_F);
         if (!exact) {
@@ -876,12 +869,6 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
           part = exp_pass((m_run == -CUDART_INF_F) ? 0.f : -m_run, false, unused);
         }
         l_run += part;
-#if SWA_SOFTMAX_PINGPONG
-        if (hpc == 2) {  // hand the sub-partition's SFU to the other head
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(bar_turn + 8 * ((1 - i) * 4 + (warp & 3)));
-        }
-#endif
         tc::tc_wait_st();
         tc::tc_fence_before();
         __syncwarp();
