@@ -2,11 +2,16 @@
 // chunk itself (Mistral 7B, section 2, Pre-fill and Chunking paragraph and
 // Figure 3), on the 5th-generation tensor cores of sm_100a.
 //
-// One CTA = one 128-row query tile of one or two query heads that share a kv
-// head (GQA: both heads reuse every K/V tile the CTA loads).  Warp roles:
+// A unit of work is one 128-row query tile of one or two query heads that
+// share a kv head (GQA: both heads reuse every K/V tile the CTA loads) of one
+// sequence.  With a workspace the grid is one CTA per SM and each CTA takes
+// units, heaviest first, from a counter in the workspace; the units of the
+// last round are cut into pieces of their key range whose partial softmax
+// results are merged by log-sum-exp.  Without one, the grid has one CTA per
+// unit.  Warp roles:
 //   warps 0-3  softmax for head slot 0 (TMEM lanes 0-127 = the 128 query rows)
 //   warps 4-7  softmax for head slot 1
-//   warp  8    TMA producer: Q once, then K tiles into an NK-stage ring
+//   warp  8    TMA producer: Q of each unit, then K tiles into an NK-stage ring
 //   warp  9    TMEM allocator and MMA issuer (one elected lane issues tcgen05.mma)
 //   warp 10    TMA producer: V tiles into an NV-stage ring
 //   warp 11    work fetcher: takes units (or pieces of units) and publishes
@@ -83,6 +88,9 @@ constexpr uint32_t kTmemCols = 512;
 // partial result slot per key-range piece (at most one per persistent CTA):
 // per head, O^T [d][128 rows] followed by the running max [128] and sum [128].
 constexpr int kMaxPersistentCtas = 256;
+// A unit of the split tail is cut into pieces only if it has at least this
+// many key tiles; lighter units go whole to their first piece.
+constexpr int kMinSplitTiles = 8;
 constexpr size_t kWsMergeOffset = 256;
 constexpr size_t kWsPartialOffset = 16384;
 static_assert(kWsMergeOffset + kMaxPersistentCtas * 8 * sizeof(int) <= kWsPartialOffset, "workspace layout");
@@ -262,6 +270,13 @@ __device__ __forceinline__ Item decode_item(const PrefillParams& p, int item) {
   if (it.rows) {
     it.plan = make_plan(it.s, it.t_lo, it.qt, p.window);
     const int w = it.plan.total();
+    if (it.np > 1 && w < kMinSplitTiles) {
+      // Too few key tiles to be worth a merge (a causal first chunk's
+      // lightest tiles): piece 0 takes the whole unit, the others nothing.
+      it.rows = it.piece == 0;
+      it.np = 1;
+      if (!it.rows) return it;
+    }
     it.j0 = (int)((long long)it.piece * w / it.np);
     it.n_tiles = (int)((long long)(it.piece + 1) * w / it.np) - it.j0;
   }
@@ -497,7 +512,15 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
           continue;
         }
         SWA_TRACE_AT(1, 1000 + it);
-        if (qi > 0) ok = tc::mbar_wait(bar_q_empty, (qi - 1) & 1, p.status);
+        if (qi > 0) {
+          // The Q buffer is still in use by the previous unit's last products:
+          // pull this unit's Q tiles into L2 meanwhile, so that their load
+          // below does not wait on HBM.
+          for (int i = 0; i < hpc; ++i)
+            for (int cb = 0; cb < C::kColBlocks; ++cb)
+              tc::tma_prefetch_4d(&maps.q, cb * C::kBoxD, I.h_first + i, I.t_lo, I.b);
+          ok = tc::mbar_wait(bar_q_empty, (qi - 1) & 1, p.status);
+        }
         if (!ok) break;
         tc::mbar_arrive_expect_tx(bar_q_full, hpc * C::kTileBytes);
         for (int i = 0; i < hpc; ++i)

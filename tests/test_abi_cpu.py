@@ -155,7 +155,9 @@ def test_python_binding_refuses_to_run_without_the_library(tmp_path, monkeypatch
 
 @pytest.mark.parametrize("B,Hq,Hkv,W,expect", [
     (1, 32, 8, 4096, (8, 1)),     # 8 pairs: a cluster of 8 streaming CTAs per pair, merged in-kernel
-    (4, 32, 8, 4096, (8, 1)),     # 32 pairs: still clustered
+    (4, 32, 8, 4096, (4, 1)),     # 32 pairs: clusters of 4, so 128 CTAs run in one wave
+    (2, 32, 8, 4096, (8, 1)),     # 16 pairs: clusters of 8 (128 CTAs)
+    (6, 32, 8, 4096, (3, 1)),     # 48 pairs: clusters of 3 (144 CTAs)
     (16, 32, 8, 4096, (1, 1)),    # 128 pairs (< 148 SMs): one streaming CTA per pair
     (24, 32, 8, 4096, (3, 2)),    # 192 pairs: floor(592 / 192) = 3 splits + combine
     (32, 32, 8, 4096, (2, 2)),    # 256 pairs: 2 splits + combine

@@ -142,6 +142,29 @@ def test_prefill_matches_oracle(B, lengths, W, chunk, Hq, Hkv, d, workspace):
     np.testing.assert_array_equal(cache_as_f64(vc), rcache.v)
 
 
+# Shapes with few units per call, so the persistent schedule cuts every unit
+# that sees at least 8 key tiles into 2-4 pieces of its key range and merges
+# them (the path a 4096-token chunk takes for its last round of units).
+SPLIT_CASES = [
+    # B, lengths,      W,    chunk, Hq, Hkv, d
+    (1, [2304],        2048, 256,   4,  2,   128),   # 4 units per call: 4 pieces each
+    (2, [3000, 2100],  2048, 512,   8,  2,   64),    # ragged batch, G = 4
+    (1, [1500],        1024, 500,   3,  3,   128),   # G = 1 (one head per CTA), chunk < W
+    (1, [700],         1024, 350,   2,  1,   16),    # d = 16
+]
+
+
+@pytest.mark.parametrize("B,lengths,W,chunk,Hq,Hkv,d", SPLIT_CASES)
+def test_prefill_split_pieces_match_oracle(B, lengths, W, chunk, Hq, Hkv, d):
+    L = max(lengths)
+    q, k, v = random_case(2000 + W + chunk + d, B, L, Hq, Hkv, d, lengths=lengths)
+    dims = mk_dims(B, Hq, Hkv, d, W)
+    got, kc, vc = gpu_chunked_prefill(dims, q, k, v, lengths, chunk, workspace=True)
+    ref, rcache = oracle.run_chunked_prefill(q, k, v, W, chunk, dims.scale, lengths=lengths)
+    assert_close(got, ref, f"split pieces B={B} L={lengths} W={W} chunk={chunk}")
+    np.testing.assert_array_equal(cache_as_f64(kc), rcache.k)
+
+
 def test_prefill_bf16_output():
     B, L, W, Hq, Hkv, d = 2, 300, 128, 8, 2, 128
     q, k, v = random_case(77, B, L, Hq, Hkv, d)
@@ -196,7 +219,7 @@ DECODE_CASES = [
     # 80 pairs: one streaming CTA per pair, 11 chunks with a partial last one,
     # caches from empty to wrapped
     (10, 700, 16, 8, 64, [0, 5, 699, 700, 1500, 33, 2000, 64, 65, 128], 2),
-    (6, 2048, 32, 8, 128, [9000, 2047, 2048, 100, 3000, 4100], 2),  # 48 pairs: clusters of 4
+    (6, 2048, 32, 8, 128, [9000, 2047, 2048, 100, 3000, 4100], 2),  # 48 pairs: clusters of 3
 ]
 
 
