@@ -48,11 +48,11 @@ METRIC = ("prefill tokens/s & TFLOP/s (% bf16 peak); decode tokens/s & HBM GB/s 
 # while the kernel source is the one that was profiled (sha256 prefix of the .cu file);
 # the summaries with the commands are under profiles/.
 PROFILED_TRAFFIC = {
-    "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "0cdc3b2e8f72bfe1",
-                           "bytes": 67_197_184 + 5_038_080,
+    "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "4ecc10552800aea3",
+                           "bytes": 67_403_776 + 12_481_536,
                            "launch": "chunk 1 of 4 (every row sees 4096 keys)"},
-    "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "7d6ddd2772e3e77d",
-                          "bytes": 1_074_303_000 + 3_859_712, "launch": "one decode step"},
+    "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "ef030e747ec614ee",
+                          "bytes": 1_074_320_000 + 3_678_720, "launch": "one decode step"},
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
