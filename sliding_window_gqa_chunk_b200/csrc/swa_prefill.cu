@@ -512,15 +512,7 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
           continue;
         }
         SWA_TRACE_AT(1, 1000 + it);
-        if (qi > 0) {
-          // The Q buffer is still in use by the previous unit's last products:
-          // pull this unit's Q tiles into L2 meanwhile, so that their load
-          // below does not wait on HBM.
-          for (int i = 0; i < hpc; ++i)
-            for (int cb = 0; cb < C::kColBlocks; ++cb)
-              tc::tma_prefetch_4d(&maps.q, cb * C::kBoxD, I.h_first + i, I.t_lo, I.b);
-          ok = tc::mbar_wait(bar_q_empty, (qi - 1) & 1, p.status);
-        }
+        if (qi > 0) ok = tc::mbar_wait(bar_q_empty, (qi - 1) & 1, p.status);
         if (!ok) break;
         tc::mbar_arrive_expect_tx(bar_q_full, hpc * C::kTileBytes);
         for (int i = 0; i < hpc; ++i)
