@@ -65,6 +65,17 @@ namespace {
   } while (0)
 #endif
 
+// Bits [lo, hi) of the 32 keys that start at key w0, as a mask.
+__device__ __forceinline__ uint32_t range_bits(int lo, int hi, int w0) {
+  int l = lo - w0, h = hi - w0;
+  l = l < 0 ? 0 : (l > 32 ? 32 : l);
+  h = h < 0 ? 0 : (h > 32 ? 32 : h);
+  if (h <= l) return 0u;
+  const uint32_t hm = h >= 32 ? 0xffffffffu : ((1u << h) - 1u);
+  const uint32_t lm = l >= 32 ? 0xffffffffu : ((1u << l) - 1u);
+  return hm & ~lm;
+}
+
 constexpr int kRows = 128;          // query rows per tile = TMEM lanes
 constexpr int kKeys = 128;          // keys per tile
 constexpr int kThreads = 384;       // 12 warps = 3 warpgroups
@@ -759,29 +770,33 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
         bool is_cache;
         int kbase;
         I.plan.at(I.j0 + j, is_cache, kbase);
+        // Visible keys of this row in this tile: [v_lo0, v_hi0) U [v_lo1, v_hi1).
+        // A cache tile: slot kbase + k is visible iff it is < W and
+        // (kbase + k - a_i) mod W < len_i, i.e. k < len_i - d0, or
+        // W - d0 <= k < W - d0 + len_i.  A chunk tile: key kbase + k <= t.
         bool masked = false;  // this row has invisible keys in this tile
+        int v_lo0 = 0, v_hi0 = kKeys, v_lo1 = 0, v_hi1 = 0;
         if (is_cache) {
           int d0 = kbase - a_i;
           if (d0 < 0) d0 += W;
           masked = !((kbase + kKeys <= W) && (len_i > 0) && (d0 + kKeys <= len_i));
-          if (masked) {
-            // slot kbase + k is visible iff it is < W and (kbase + k - a_i) mod W
-            // < len_i, i.e. k < len_i - d0, or W - d0 <= k < W - d0 + len_i
-            const int a_end = len_i - d0, b_lo = W - d0, b_end = W - d0 + len_i;
-            const int r_end = W - kbase;
-#pragma unroll
-            for (int k = 0; k < kKeys; ++k) {
-              const bool vis = (k < a_end || (k >= b_lo && k < b_end)) && k < r_end;
-              if (!vis) sv[k] = -CUDART_INF_F;
-            }
-          }
+          const int r_end = W - kbase;
+          v_hi0 = min(len_i - d0, r_end);
+          v_lo1 = W - d0;
+          v_hi1 = min(W - d0 + len_i, r_end);
         } else {
           masked = kbase + kKeys - 1 > t;
-          if (masked) {
+          v_hi0 = t - kbase + 1;
+        }
+        if (masked) {
+          // as four 32-bit visibility words, then one select per score
+          uint32_t vm[kKeys / 32];
 #pragma unroll
-            for (int k = 0; k < kKeys; ++k)
-              if (kbase + k > t) sv[k] = -CUDART_INF_F;
-          }
+          for (int w = 0; w < kKeys / 32; ++w)
+            vm[w] = range_bits(v_lo0, v_hi0, 32 * w) | range_bits(v_lo1, v_hi1, 32 * w);
+#pragma unroll
+          for (int k = 0; k < kKeys; ++k)
+            sv[k] = ((vm[k >> 5] >> (k & 31)) & 1u) ? sv[k] : -CUDART_INF_F;
         }
 #ifdef SWA_TILE_COUNTERS
         {  // checked build: (warp, tile) pairs with / without a masked key
