@@ -675,11 +675,13 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
             if (!ok) break;
           }
           const int svp = vt % NV;
+          // V(j - 1) is checked while the softmax of tile j - 1 still runs, so
+          // that the P V products follow the P-ready arrivals directly.
+          if (j > 0)
+            ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_v_full + 8 * svp, (vt / NV) & 1, p.status));
           for (int i = 0; i < hpc && ok; ++i) {
             if (j > 0) {
               ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_p_full + 8 * i, (g0 + j - 1) & 1, p.status));
-              if (ok && i == 0)
-                ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_v_full + 8 * svp, (vt / NV) & 1, p.status));
               if (!ok) break;
               tc::tc_fence_after();
               issue_pv(i, svp, j - 1 > 0);
