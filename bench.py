@@ -48,8 +48,8 @@ METRIC = ("prefill tokens/s & TFLOP/s (% bf16 peak); decode tokens/s & HBM GB/s 
 # while the kernel source is the one that was profiled (sha256 prefix of the .cu file);
 # the summaries with the commands are under profiles/.
 PROFILED_TRAFFIC = {
-    "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "b8f545d605e00baa",
-                           "bytes": 67_340_800 + 11_744_768,
+    "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "1ecd2f622b8ca9b0",
+                           "bytes": 67_265_280 + 11_899_904,
                            "launch": "chunk 1 of 4 (every row sees 4096 keys)"},
     "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "ef030e747ec614ee",
                           "bytes": 1_074_320_000 + 3_678_720, "launch": "one decode step"},
