@@ -274,7 +274,22 @@ namespace swa {
 #define SWA_DECODE_SPLIT_FLOOR 1
 #endif
 
-DecodeSplit decode_split(int batch, int n_q_heads, int n_kv_heads, int window) {
+namespace {
+
+// Resident clusters of the d = 128 stream-variant decode CTA (one per SM: a
+// 192 KiB ring) on a 148-SM B200, as cudaOccupancyMaxActiveClusters reports
+// them (index = cluster size): the SMs of a cluster share a GPC, so larger
+// clusters leave SMs unused.  Used only where no device can be asked.
+constexpr int kB200ResidentClusters[9] = {0, 148, 74, 45, 33, 26, 22, 15, 15};
+
+int resident_clusters(int head_dim, int cs) {
+  const int n = decode_resident_clusters(head_dim, cs);
+  return n >= 0 ? n : kB200ResidentClusters[cs];
+}
+
+}  // namespace
+
+DecodeSplit decode_split(int batch, int n_q_heads, int n_kv_heads, int window, int head_dim) {
   const long long units = (long long)batch * n_kv_heads;
   // Workspace split: about four resident 128-thread CTAs per SM on a 148-SM
   // B200, each split a multiple of 64 slots (16 per warp); the per-split fp32
@@ -322,6 +337,10 @@ DecodeSplit decode_split(int batch, int n_q_heads, int n_kv_heads, int window) {
       if (cs > kDecodeMaxClusterSplits) cs = kDecodeMaxClusterSplits;
       if (cs > 148 / units) cs = 148 / units;
       if (cs < 1) cs = 1;
+      // All clusters of the launch must be resident at once (a second wave
+      // nearly doubles the step): shrink the cluster until the device holds
+      // one per pair.
+      while (cs > 1 && units > resident_clusters(head_dim, (int)cs)) --cs;
     }
     long long cper = (window + cs - 1) / cs;
     cper = (cper + 15) / 16 * 16;
@@ -444,7 +463,7 @@ int swa_prefill_chunk(const swa_dims* dims, void* out, const void* q, const void
 size_t swa_decode_workspace_size(const swa_dims* dims) {
   if (check_dims(dims) != SWA_OK) return 0;
   const swa::DecodeSplit sp =
-      swa::decode_split(dims->batch, dims->n_q_heads, dims->n_kv_heads, dims->window);
+      swa::decode_split(dims->batch, dims->n_q_heads, dims->n_kv_heads, dims->window, dims->head_dim);
   if (sp.ws_splits <= 1) return 16;  // nothing needed; a non-zero size keeps callers simple
   const size_t bh = (size_t)dims->batch * dims->n_q_heads * sp.ws_splits;
   return bh * dims->head_dim * sizeof(float) + bh * 2 * sizeof(float);
@@ -454,7 +473,7 @@ int swa_decode_launch_info(const swa_dims* dims, int32_t* n_splits, int32_t* n_l
   int rc = check_dims(dims);
   if (rc) return rc;
   const swa::DecodeSplit sp =
-      swa::decode_split(dims->batch, dims->n_q_heads, dims->n_kv_heads, dims->window);
+      swa::decode_split(dims->batch, dims->n_q_heads, dims->n_kv_heads, dims->window, dims->head_dim);
   if (n_splits) *n_splits = sp.n_splits;
   // a cluster merges its splits in-kernel; otherwise several splits need the combine kernel
   if (n_launches) *n_launches = (sp.n_splits > 1 && !sp.cluster) ? 2 : 1;
@@ -477,7 +496,7 @@ int swa_decode(const swa_dims* dims, void* out, const void* q, const void* k_new
   int* status = nullptr;
   if ((rc = status_ptr(&status))) return rc;
   const swa::DecodeSplit sp =
-      swa::decode_split(dims->batch, dims->n_q_heads, dims->n_kv_heads, dims->window);
+      swa::decode_split(dims->batch, dims->n_q_heads, dims->n_kv_heads, dims->window, dims->head_dim);
   swa::DecodeParams p;
   p.out = out;
   p.q = static_cast<const __nv_bfloat16*>(q);

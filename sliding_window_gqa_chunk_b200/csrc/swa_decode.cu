@@ -188,6 +188,18 @@ constexpr int kStreamStages = 6;
 template <int D>
 constexpr int stream_ring_bytes() { return kStreamStages * 2 * kChunkSlots * D * 2; }
 
+// Row stride (floats) of the per-warp O partials in shared memory: one float
+// of padding spreads the rows that a warp's lanes store at once over the banks
+// (with stride D the 4 head rows and the two halves of the d range would all
+// land on the same 4 banks).
+template <int D>
+constexpr int merge_o_stride() { return D + 1; }
+// Shared memory of the CTA merge: m, l and O of each warp, then the CTA's m, l, O.
+template <int D, int NT, int NW>
+constexpr int decode_merge_bytes() {
+  return (int)sizeof(float) * (NW * 8 * NT * (2 + merge_o_stride<D>()) + 8 * NT * (2 + D));
+}
+
 // Programmatic dependent launch: the kernels below are launched with
 // programmatic stream serialization, so they may be scheduled while the
 // previous kernel in the stream is still running; this wait (first thing in
@@ -267,7 +279,8 @@ swa_decode_kernel(const DecodeParams p) {
 
   // ---- stream variant: ring of K / V chunks, full / empty barriers ----
   constexpr int G8 = 8 * NT;
-  constexpr int kMergeBytes = (int)sizeof(float) * (NW + 1) * G8 * (2 + D);
+  constexpr int kMergeBytes = decode_merge_bytes<D, NT, NW>();
+  constexpr int kOS = merge_o_stride<D>();
   constexpr int kRingBytes = STREAM ? stream_ring_bytes<D>() : 0;
   constexpr int kBarOffset = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
   const uint32_t s_base = tc::smem_u32(smem);
@@ -438,7 +451,7 @@ swa_decode_kernel(const DecodeParams p) {
   }
 
   // ---- merge the NW warps of the CTA ----
-  // smem: m[NW][G8], l[NW][G8], O[NW][G8][D] with G8 = 8*NT, then the CTA's
+  // smem: m[NW][G8], l[NW][G8], O[NW][G8][kOS] with G8 = 8*NT, then the CTA's
   // partial m[G8], l[G8], O[G8][D] (cluster merge); in the stream variant this
   // reuses the ring, once every warp is done with it.
   if constexpr (STREAM) {
@@ -448,7 +461,7 @@ swa_decode_kernel(const DecodeParams p) {
   float* sm_m = smem;
   float* sm_l = sm_m + NW * G8;
   float* sm_o = sm_l + NW * G8;
-  float* cta_m = sm_o + (size_t)NW * G8 * D;
+  float* cta_m = sm_o + (size_t)NW * G8 * kOS;
   float* cta_l = cta_m + G8;
   float* cta_o = cta_l + G8;
 #pragma unroll
@@ -475,8 +488,8 @@ swa_decode_kernel(const DecodeParams p) {
       } else {
         d0 = (mt / 4) * 64 + g * 8 + (mt % 4) * 2;
       }
-      float* oh0 = sm_o + ((size_t)warp * G8 + h0) * D;
-      float* oh1 = oh0 + D;
+      float* oh0 = sm_o + ((size_t)warp * G8 + h0) * kOS;
+      float* oh1 = oh0 + kOS;
       oh0[d0] = o[nt][mt][0];
       oh1[d0] = o[nt][mt][1];
       oh0[d0 + 1] = o[nt][mt][2];
@@ -498,7 +511,7 @@ swa_decode_kernel(const DecodeParams p) {
       for (int w = 0; w < NW; ++w) {
         const float sc = fast_exp2(sm_m[w * G8 + h] - M);
         L += sc * sm_l[w * G8 + h];
-        O += sc * sm_o[((size_t)w * G8 + h) * D + dd];
+        O += sc * sm_o[((size_t)w * G8 + h) * kOS + dd];
       }
     }
     const size_t bh = (size_t)b * p.n_q_heads + hq0 + h;
@@ -598,8 +611,7 @@ constexpr int kMaxDevices = 64;
 
 template <int D, int NT, int NW, typename OutT, bool STREAM>
 cudaError_t launch_decode_t(const DecodeParams& p, cudaStream_t stream) {
-  constexpr int G8 = 8 * NT;
-  constexpr size_t merge = sizeof(float) * (size_t)(NW + 1) * G8 * (2 + D);
+  constexpr size_t merge = (size_t)decode_merge_bytes<D, NT, NW>();
   constexpr size_t ring = STREAM ? (size_t)stream_ring_bytes<D>() : 0;
   constexpr size_t smem = (ring > merge ? ring : merge) + (STREAM ? 16 * kStreamStages : 0);
   auto kern = swa_decode_kernel<D, NT, NW, OutT, STREAM>;
@@ -663,7 +675,58 @@ cudaError_t launch_decode_o(const DecodeParams& p, cudaStream_t stream) {
   return cudaErrorInvalidValue;
 }
 
+template <int D>
+int resident_clusters_d(int cs) {
+  auto kern = swa_decode_kernel<D, 1, 8, __nv_bfloat16, true>;
+  constexpr size_t merge = (size_t)decode_merge_bytes<D, 1, 8>();
+  constexpr size_t ring = (size_t)stream_ring_bytes<D>();
+  constexpr size_t smem = (ring > merge ? ring : merge) + 16 * kStreamStages;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return -1;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)cs);
+  cfg.blockDim = dim3(9 * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) return -1;
+  return n;
+}
+
 }  // namespace
+
+int decode_resident_clusters(int head_dim, int cs) {
+  if (cs < 1 || cs > kDecodeMaxClusterSplits) return -1;
+  const int di = head_dim == 16 ? 0 : head_dim == 64 ? 1 : head_dim == 128 ? 2 : -1;
+  int dev = 0;
+  if (di < 0 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();  // no device: leave no error behind for the next call
+    return -1;
+  }
+  // answers per device, head dimension and cluster size (value + 1; 0 = not asked yet)
+  static int cache[kMaxDevices][3][kDecodeMaxClusterSplits + 1] = {};
+  int& c = cache[dev][di][cs];
+  if (c == 0) {
+    int n = -1;
+    switch (head_dim) {
+      case 16: n = resident_clusters_d<16>(cs); break;
+      case 64: n = resident_clusters_d<64>(cs); break;
+      default: n = resident_clusters_d<128>(cs); break;
+    }
+    if (n < 0) {
+      cudaGetLastError();
+      return -1;
+    }
+    c = n + 1;
+  }
+  return c - 1;
+}
 
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream) {
   if (p.out_f32) return launch_decode_o<float>(p, stream);

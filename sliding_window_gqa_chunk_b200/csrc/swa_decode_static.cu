@@ -88,7 +88,7 @@ extern "C" SWA_API int swa_decode_static(const swa_dims* dims, void* out, const 
   // or a thread-block cluster merges the splits, else one fp32 partial
   // (d values, max and sum) per (sequence, query head, split).
   const swa::DecodeSplit sp =
-      swa::decode_split(dims->batch, dims->n_q_heads, dims->n_kv_heads, dims->window);
+      swa::decode_split(dims->batch, dims->n_q_heads, dims->n_kv_heads, dims->window, dims->head_dim);
   const size_t bh = (size_t)dims->batch * dims->n_q_heads * sp.n_splits;
   const size_t need = (sp.cluster || sp.n_splits == 1) ? 0 : bh * (dims->head_dim + 2) * sizeof(float);
   if (need > kStaticScratchBytes)

@@ -58,7 +58,12 @@ struct DecodeSplit {
   int stream;
   int ws_splits;   // splits the workspace is sized for (fp32 partials per split)
 };
-DecodeSplit decode_split(int batch, int n_q_heads, int n_kv_heads, int window);
+DecodeSplit decode_split(int batch, int n_q_heads, int n_kv_heads, int window, int head_dim);
+
+// Thread-block clusters of `cs` stream-variant decode CTAs (head dimension
+// head_dim) that the current device holds at once, or -1 when it cannot be
+// asked (no device).
+int decode_resident_clusters(int head_dim, int cs);
 
 struct PrefillParams {
   void* out;                    // [B][max_tokens][Hq][d] bf16 or f32

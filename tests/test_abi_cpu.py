@@ -156,8 +156,9 @@ def test_python_binding_refuses_to_run_without_the_library(tmp_path, monkeypatch
 @pytest.mark.parametrize("B,Hq,Hkv,W,expect", [
     (1, 32, 8, 4096, (8, 1)),     # 8 pairs: a cluster of 8 streaming CTAs per pair, merged in-kernel
     (4, 32, 8, 4096, (4, 1)),     # 32 pairs: clusters of 4, so 128 CTAs run in one wave
-    (2, 32, 8, 4096, (8, 1)),     # 16 pairs: clusters of 8 (128 CTAs)
-    (6, 32, 8, 4096, (3, 1)),     # 48 pairs: clusters of 3 (144 CTAs)
+    (2, 32, 8, 4096, (6, 1)),     # 16 pairs: a B200 holds 15 clusters of 8 or 7, 22 of 6
+    (3, 32, 8, 4096, (5, 1)),     # 24 pairs: 22 clusters of 6 fit, 26 of 5
+    (6, 32, 8, 4096, (2, 1)),     # 48 pairs: 45 clusters of 3 fit, 74 of 2
     (16, 32, 8, 4096, (1, 1)),    # 128 pairs (< 148 SMs): one streaming CTA per pair
     (24, 32, 8, 4096, (3, 2)),    # 192 pairs: floor(592 / 192) = 3 splits + combine
     (32, 32, 8, 4096, (2, 2)),    # 256 pairs: 2 splits + combine
@@ -168,6 +169,8 @@ def test_python_binding_refuses_to_run_without_the_library(tmp_path, monkeypatch
     (3, 12, 4, 100, (1, 1)),
 ])
 def test_decode_launch_info_follows_the_split_rule(B, Hq, Hkv, W, expect):
+    # Without a device the cluster sizes come from the resident-cluster counts
+    # of a 148-SM B200 (on a GPU the library asks the device itself).
     d = swa.Dims(B, Hq, Hkv, 128, W, 0.1, "bf16")
     assert swa.decode_launch_info(d) == expect
 

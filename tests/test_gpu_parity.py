@@ -219,7 +219,11 @@ DECODE_CASES = [
     # 80 pairs: one streaming CTA per pair, 11 chunks with a partial last one,
     # caches from empty to wrapped
     (10, 700, 16, 8, 64, [0, 5, 699, 700, 1500, 33, 2000, 64, 65, 128], 2),
-    (6, 2048, 32, 8, 128, [9000, 2047, 2048, 100, 3000, 4100], 2),  # 48 pairs: clusters of 3
+    (6, 2048, 32, 8, 128, [9000, 2047, 2048, 100, 3000, 4100], 2),  # 48 pairs: clusters of 2
+    # clusters sized so that every pair's cluster is resident at once: 16 pairs
+    # take clusters of 6 (688 slots per CTA, 656 in the last), 24 pairs of 5
+    (2, 4096, 32, 8, 128, [50000, 4097], 2),
+    (3, 4096, 32, 8, 128, [4096, 12345, 700], 2),
 ]
 
 
