@@ -188,6 +188,13 @@ constexpr int kStreamStages = 6;
 template <int D>
 constexpr int stream_ring_bytes() { return kStreamStages * 2 * kChunkSlots * D * 2; }
 
+// Compute warps of the stream variant (one more warp streams the ring).
+// Warp w takes the 16-slot blocks w, w + NW, ... of its split, so it reads
+// every (NW / 4)-th chunk; that stride must divide the stage count, or a warp
+// could skip a fill of a stage and take a later fill's parity for an earlier
+// one.  12 warps: chunks 3 apart, 2 stages per warp.
+constexpr int kStreamWarps = 12;
+
 // Row stride (floats) of the per-warp O partials in shared memory: one float
 // of padding spreads the rows that a warp's lanes store at once over the banks
 // (with stride D the 4 head rows and the two halves of the d range would all
@@ -278,6 +285,9 @@ swa_decode_kernel(const DecodeParams p) {
   }
 
   // ---- stream variant: ring of K / V chunks, full / empty barriers ----
+  static_assert(!STREAM || ((NW * kBlockSlots) % kChunkSlots == 0 &&
+                            kStreamStages % (NW * kBlockSlots / kChunkSlots) == 0),
+                "a compute warp must see every fill of each ring stage it reads");
   constexpr int G8 = 8 * NT;
   constexpr int kMergeBytes = decode_merge_bytes<D, NT, NW>();
   constexpr int kOS = merge_o_stride<D>();
@@ -658,8 +668,8 @@ template <int D, typename OutT>
 cudaError_t launch_decode_d(const DecodeParams& p, cudaStream_t stream) {
   const int G = p.n_q_heads / p.n_kv_heads;
   if (p.stream) {
-    if (G <= 8) return launch_decode_t<D, 1, 8, OutT, true>(p, stream);
-    return launch_decode_t<D, 2, 8, OutT, true>(p, stream);
+    if (G <= 8) return launch_decode_t<D, 1, kStreamWarps, OutT, true>(p, stream);
+    return launch_decode_t<D, 2, kStreamWarps, OutT, true>(p, stream);
   }
   if (G <= 8) return launch_decode_t<D, 1, 4, OutT, false>(p, stream);
   return launch_decode_t<D, 2, 4, OutT, false>(p, stream);
@@ -677,8 +687,8 @@ cudaError_t launch_decode_o(const DecodeParams& p, cudaStream_t stream) {
 
 template <int D>
 int resident_clusters_d(int cs) {
-  auto kern = swa_decode_kernel<D, 1, 8, __nv_bfloat16, true>;
-  constexpr size_t merge = (size_t)decode_merge_bytes<D, 1, 8>();
+  auto kern = swa_decode_kernel<D, 1, kStreamWarps, __nv_bfloat16, true>;
+  constexpr size_t merge = (size_t)decode_merge_bytes<D, 1, kStreamWarps>();
   constexpr size_t ring = (size_t)stream_ring_bytes<D>();
   constexpr size_t smem = (ring > merge ? ring : merge) + 16 * kStreamStages;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
@@ -690,7 +700,7 @@ int resident_clusters_d(int cs) {
   attr[0].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)cs);
-  cfg.blockDim = dim3(9 * 32);
+  cfg.blockDim = dim3((kStreamWarps + 1) * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
