@@ -324,13 +324,14 @@ DecodeSplit decode_split(int batch, int n_q_heads, int n_kv_heads, int window, i
   if (units < 148) {
     // Fewer (sequence, kv head) pairs than SMs: one launch of CTAs whose
     // producer warp streams the split's slots into shared memory with bulk
-    // copies, so every byte of a split is in flight at once.  Below 64 pairs
-    // the window of a pair is split over a thread-block cluster of up to 8
-    // CTAs (about 512 slots each, no more CTAs than SMs) that merge through
-    // distributed shared memory; from 64 pairs on one CTA covers a pair's
-    // whole window.  No workspace and no combine kernel either way.
+    // copies, so every byte of a split is in flight at once.  The window of
+    // a pair is split over a thread-block cluster of up to 8 CTAs (about 512
+    // slots each, no more CTAs than SMs) that merge through distributed
+    // shared memory; from 75 pairs on (a B200 holds 74 clusters of 2) one
+    // CTA covers a pair's whole window.  No workspace and no combine kernel
+    // either way.
     long long cs = 1;
-    if (units < 64) {
+    {
       // at most one CTA per SM in all (each holds a 192 KiB ring), so the
       // clusters of a launch run in one wave
       cs = (window + 511) / 512;

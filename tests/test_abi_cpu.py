@@ -159,6 +159,9 @@ def test_python_binding_refuses_to_run_without_the_library(tmp_path, monkeypatch
     (2, 32, 8, 4096, (6, 1)),     # 16 pairs: a B200 holds 15 clusters of 8 or 7, 22 of 6
     (3, 32, 8, 4096, (5, 1)),     # 24 pairs: 22 clusters of 6 fit, 26 of 5
     (6, 32, 8, 4096, (2, 1)),     # 48 pairs: 45 clusters of 3 fit, 74 of 2
+    (8, 32, 8, 4096, (2, 1)),     # 64 pairs: clusters of 2 (74 fit)
+    (9, 32, 8, 4096, (2, 1)),     # 72 pairs: clusters of 2
+    (10, 32, 8, 4096, (1, 1)),    # 80 pairs: no room for clusters of 2, one CTA per pair
     (16, 32, 8, 4096, (1, 1)),    # 128 pairs (< 148 SMs): one streaming CTA per pair
     (24, 32, 8, 4096, (3, 2)),    # 192 pairs: floor(592 / 192) = 3 splits + combine
     (32, 32, 8, 4096, (2, 2)),    # 256 pairs: 2 splits + combine

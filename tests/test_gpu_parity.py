@@ -224,6 +224,8 @@ DECODE_CASES = [
     # take clusters of 6 (688 slots per CTA, 656 in the last), 24 pairs of 5
     (2, 4096, 32, 8, 128, [50000, 4097], 2),
     (3, 4096, 32, 8, 128, [4096, 12345, 700], 2),
+    # 64 pairs: clusters of 2 (2048 slots each)
+    (8, 4096, 32, 8, 128, [4096, 9000, 100, 4095, 20000, 7000, 1, 5000], 2),
 ]
 
 
