@@ -51,8 +51,8 @@ PROFILED_TRAFFIC = {
     "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "1ecd2f622b8ca9b0",
                            "bytes": 67_265_280 + 11_899_904,
                            "launch": "chunk 1 of 4 (every row sees 4096 keys)"},
-    "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "ef030e747ec614ee",
-                          "bytes": 1_074_320_000 + 3_678_720, "launch": "one decode step"},
+    "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "162841c6a1d30b0e",
+                          "bytes": 1_074_293_248 + 3_966_976, "launch": "one decode step"},
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
@@ -770,7 +770,7 @@ def main(argv=None):
                     default="all",
                     help="run one phase only (for profiling); the headline line needs 'all'")
     ap.add_argument("--batches", type=lambda x: [int(b) for b in x.split(",")],
-                    default=[1, 16, 64, 128],
+                    default=[1, 4, 8, 16, 64, 128],
                     help="batch sizes of the 32-layer decode phase (comma list)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
