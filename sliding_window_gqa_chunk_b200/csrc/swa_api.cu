@@ -455,6 +455,8 @@ int swa_prefill_chunk(const swa_dims* dims, void* out, const void* q, const void
   p.workspace = workspace;
   p.scale_log2 = dims->scale * 1.4426950408889634f;
   p.out_f32 = dims->out_dtype == SWA_DTYPE_F32;
+  // every row and 16-element piece of a row starts 32 bytes apart from the base
+  p.out_v8 = (reinterpret_cast<uintptr_t>(out) % 32) == 0;
   p.trace = g_trace;
   e = swa::launch_prefill(p, maps, (int)sc.grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "swa_prefill_chunk launch");

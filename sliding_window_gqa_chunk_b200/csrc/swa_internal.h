@@ -79,6 +79,7 @@ struct PrefillParams {
   int persistent;               // 1: CTAs take items from the workspace counter
   float scale_log2;
   int out_f32;
+  int out_v8;                   // 1: out is 32-byte aligned (the epilogue stores 32 bytes per instruction)
   void* workspace;              // caller scratch (NULL: no key-range splits)
   int* trace;                   // progress words in host-mapped memory (trace builds only)
 };

@@ -194,10 +194,27 @@ __device__ __forceinline__ TilePlan make_plan(long long s, int t_lo, int qt, int
 }
 
 template <typename OutT>
-__device__ __forceinline__ void store16(OutT* dst, const float (&v)[16], float scale);
+__device__ __forceinline__ void store16(OutT* dst, const float (&v)[16], float scale, bool v8);
+
+// 32 bytes in one instruction (sm_100 256-bit store); dst must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* dst, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst), "r"(w[0]), "r"(w[1]),
+               "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
 
 template <>
-__device__ __forceinline__ void store16<float>(float* dst, const float (&v)[16], float scale) {
+__device__ __forceinline__ void store16<float>(float* dst, const float (&v)[16], float scale, bool v8) {
+  if (v8) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      uint32_t w[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w[e] = __float_as_uint(v[8 * i + e] * scale);
+      st_global_v8(dst + 8 * i, w);
+    }
+    return;
+  }
   float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
   for (int i = 0; i < 4; ++i)
@@ -207,17 +224,17 @@ __device__ __forceinline__ void store16<float>(float* dst, const float (&v)[16],
 
 template <>
 __device__ __forceinline__ void store16<__nv_bfloat16>(__nv_bfloat16* dst, const float (&v)[16],
-                                                       float scale) {
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
+                                                       float scale, bool v8) {
+  uint32_t w[8];
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    uint4 w;
-    w.x = pack_bf16x2(v[8 * i + 0] * scale, v[8 * i + 1] * scale);
-    w.y = pack_bf16x2(v[8 * i + 2] * scale, v[8 * i + 3] * scale);
-    w.z = pack_bf16x2(v[8 * i + 4] * scale, v[8 * i + 5] * scale);
-    w.w = pack_bf16x2(v[8 * i + 6] * scale, v[8 * i + 7] * scale);
-    d4[i] = w;
+  for (int e = 0; e < 8; ++e) w[e] = pack_bf16x2(v[2 * e] * scale, v[2 * e + 1] * scale);
+  if (v8) {
+    st_global_v8(dst, w);
+    return;
   }
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+  d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
 
@@ -932,13 +949,19 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
                   (((size_t)I.b * p.max_tokens + t) * p.n_q_heads + (I.h_first + i)) * D;
       if (I.np == 1) {
         const float inv_l = 1.f / l_run;
+        // the whole row of O in one batch of loads and one wait
+        float ov[D];
 #pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-          float ov[16];
-          tc::tmem_ld16(tO + c * 16, ov);
-          tc::tc_wait_ld();
-          tc::reg_fence16(ov);
-          if (t < I.n) store16<OutT>(dst + c * 16, ov, inv_l);
+        for (int c = 0; c < D / 16; ++c)
+          tc::tmem_ld16(tO + c * 16, *reinterpret_cast<float(*)[16]>(ov + c * 16));
+        tc::tc_wait_ld();
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) tc::reg_fence16(ov + c * 16);
+        if (t < I.n) {
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c)
+            store16<OutT>(dst + c * 16, *reinterpret_cast<const float(*)[16]>(ov + c * 16), inv_l,
+                          p.out_v8 != 0);
         }
         continue;
       }
@@ -1017,7 +1040,7 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
             for (int e = 0; e < 16; ++e) ov[e] += a_q[q] * ld_cg(pq + e * kRows);
           }
         }
-        if (t < I.n) store16<OutT>(dst + c * 16, ov, inv_l);
+        if (t < I.n) store16<OutT>(dst + c * 16, ov, inv_l, p.out_v8 != 0);
       }
     }
     if (row == 0) SWA_TRACE_AT(3 + i, ok ? 8000 : 7500);

@@ -174,6 +174,38 @@ def test_prefill_bf16_output():
     assert_close(got, ref, "bf16 out", bf16_out=True)
 
 
+@pytest.mark.parametrize("out_dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_output_16_byte_aligned(out_dtype, d):
+    """The epilogue stores 32 bytes per instruction when the output base is
+    32-byte aligned, 16 otherwise: an output 16 bytes past a 32-byte boundary
+    gets the same values, bit for bit."""
+    B, L, W, Hq, Hkv = 2, 256, 256, 8, 2
+    q, k, v = random_case(4242 + d, B, L, Hq, Hkv, d)
+    dims = mk_dims(B, Hq, Hkv, d, W, out=out_dtype)
+    kc_a, vc_a = swa.new_cache(dims, DEV)
+    kc_b, vc_b = swa.new_cache(dims, DEV)
+    qg, kg, vg = q.to(DEV), k.to(DEV), v.to(DEV)
+    sp, nt = dev_i32([0] * B), dev_i32([L] * B)
+    n = B * L * Hq * d
+    shift = 16 // torch.empty((), dtype=dims.torch_out_dtype).element_size()
+    buf = torch.full((n + 64,), float("nan"), dtype=dims.torch_out_dtype, device=DEV)
+    base = (-buf.data_ptr() % 32) // buf.element_size()       # first 32-byte-aligned element
+    out_a = buf[base:base + n].view(B, L, Hq, d)
+    buf_b = torch.full((n + 64,), float("nan"), dtype=dims.torch_out_dtype, device=DEV)
+    off = (-buf_b.data_ptr() % 32) // buf_b.element_size() + shift
+    out_b = buf_b[off:off + n].view(B, L, Hq, d)
+    assert out_a.data_ptr() % 32 == 0 and out_b.data_ptr() % 32 == 16
+    swa.prefill_chunk(dims, out_a, qg, kg, vg, kc_a, vc_a, sp, nt)
+    swa.prefill_chunk(dims, out_b, qg, kg, vg, kc_b, vc_b, sp, nt)
+    torch.cuda.synchronize()
+    swa.device_status()
+    assert torch.equal(out_a, out_b)
+    ref, _ = oracle.run_chunked_prefill(q, k, v, W, L, dims.scale)
+    assert_close(out_b.double().cpu().numpy(), ref, f"16-byte aligned out {out_dtype} d={d}",
+                 bf16_out=out_dtype == "bf16")
+
+
 def test_prefill_chunk_after_decode_steps():
     """A chunk that starts at a position that is not a multiple of 128, after a
     few decode steps, with a cache that is not full yet (unwritten slots are zero)."""
