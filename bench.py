@@ -14,8 +14,9 @@ Alongside, in the same run and with the same step count:
   dense    - the same 16384-token inputs as one causal chunk (W = 16384): the
              "vanilla attention" side of the pages' 2x SWA claim
 Each reports its kernel's roofline fraction.  Timing: CUDA events on the
-launching stream, L2 flushed (256 MiB write) before every timed step, max over
-ranks.  Under torchrun every rank runs its own replica of the workload (the
+launching stream, L2 flushed before every timed step (a 256 MiB write, then a
+256 MiB read of another buffer so that the write's dirty lines go back to HBM
+before the step), max over ranks.  Under torchrun every rank runs its own replica of the workload (the
 path needs no exchange between GPUs), so `value` is the sum over ranks.
 
 --impl reference times the float64 CPU oracle on the same workload and prints
@@ -56,6 +57,8 @@ PROFILED_TRAFFIC = {
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
+L2_NOTE = ("flushed before every timed step (outside the timed interval): a 256 MiB write, "
+           "then a 256 MiB read of another buffer that writes the flush's dirty lines back")
 
 
 # ----------------------------------------------------------------------------
@@ -213,7 +216,7 @@ def profiled_traffic(kernel: str):
 def headline_config(wl, world: int) -> dict:
     return {"workload": wl.name, "batch": 1, "seq_len": wl.lengths[0], "window": wl.shape.window,
             "chunk": wl.chunk, "n_q_heads": 32, "n_kv_heads": 8, "head_dim": 128,
-            "out_dtype": "bf16", "l2": "flushed (256 MiB write) before every timed step",
+            "out_dtype": "bf16", "l2": L2_NOTE,
             "parallelism": f"replicas x{world}"}
 
 
@@ -510,10 +513,15 @@ def bench_ours(args, world, rank, local):
     dev = f"cuda:{local}"
     peaks = load_peaks()
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    evict_buf = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
     phase = args.phase
 
     def flush():
+        # a write larger than L2 evicts everything; reading another buffer
+        # larger than L2 then evicts the dirty lines of that write, so their
+        # write-back to HBM happens here and not inside the next timed step
         flush_buf.fill_(1)
+        evict_buf.max()
 
     wl = PREFILL_16K
     line = {
