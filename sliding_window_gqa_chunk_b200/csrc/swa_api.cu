@@ -371,6 +371,8 @@ int swa_cache_append(const swa_dims* dims, void* k_cache, void* v_cache, const v
   if ((rc = check_int_ptrs("start_pos, n_tokens", {start_pos, n_tokens}))) return rc;
   if (max_tokens < 1 || max_tokens > dims->window)
     return fail(SWA_ERR_INVALID_ARG, "max_tokens %d not in [1, window=%d]", max_tokens, dims->window);
+  if ((long long)max_tokens * dims->n_kv_heads * (dims->head_dim / 8) >= (1LL << 31))
+    return fail(SWA_ERR_UNSUPPORTED, "max_tokens * Hkv * d / 8 must stay below 2^31");
   int* status = nullptr;
   if ((rc = status_ptr(&status))) return rc;
   swa::AppendParams p;

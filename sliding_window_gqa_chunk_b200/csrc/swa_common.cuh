@@ -10,6 +10,23 @@
 
 namespace swa {
 
+// Programmatic dependent launch: the library's kernels are launched with
+// programmatic stream serialization, so they may be scheduled while the
+// previous kernel in the stream is still running; this wait (before a kernel
+// reads or writes any global memory) returns once that kernel has completed
+// and its memory writes are visible, which keeps ordinary stream order for
+// everything they read or write.  Only the launch latency and the kernel's
+// own set-up are overlapped.
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the next kernel in the stream (launched with programmatic stream
+// serialization) be scheduled onto free SMs now instead of at this kernel's
+// end; it still waits in wait_prior_grid for this kernel to complete.  Issued
+// right after this kernel's own wait, so at most one kernel runs ahead.
+__device__ __forceinline__ void allow_next_grid() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Status word codes written by kernels (first error wins).
 __device__ __forceinline__ void raise_status(int* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);

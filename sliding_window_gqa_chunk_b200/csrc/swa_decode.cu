@@ -207,21 +207,6 @@ constexpr int decode_merge_bytes() {
   return (int)sizeof(float) * (NW * 8 * NT * (2 + merge_o_stride<D>()) + 8 * NT * (2 + D));
 }
 
-// Programmatic dependent launch: the kernels below are launched with
-// programmatic stream serialization, so they may be scheduled while the
-// previous kernel in the stream is still running; this wait (first thing in
-// each kernel) returns once that kernel has completed and its memory writes
-// are visible, which keeps ordinary stream order for everything they read or
-// write.  Only the launch latency is overlapped.
-__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
-// Lets the next kernel in the stream (launched with programmatic stream
-// serialization) be scheduled onto free SMs now instead of at this kernel's
-// end; it still waits in wait_prior_grid for this kernel to complete.  Issued
-// right after this kernel's own wait, so at most one kernel runs ahead.
-__device__ __forceinline__ void allow_next_grid() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
 
 template <typename OutT>
 __device__ __forceinline__ void store_out(OutT* dst, float x);

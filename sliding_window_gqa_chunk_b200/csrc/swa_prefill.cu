@@ -459,6 +459,11 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) SWA_TRACE_AT(0, 3);
+  // Launched with programmatic stream serialization: the set-up above (no
+  // global memory) may overlap the previous kernel; nothing below reads or
+  // writes global memory before that kernel has completed.
+  wait_prior_grid();
+  allow_next_grid();
 
   // Item queue: the fetcher warp takes items (the CTA's own index first, then
   // from the shared counter when the grid is persistent), skips units with no
@@ -1094,8 +1099,17 @@ cudaError_t launch_prefill_t(const PrefillParams& p, const PrefillMaps& maps, in
     if (e != cudaSuccess) return e;
     smem_set[device] = true;
   }
-  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(p, maps);
-  return cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p, maps);
 }
 
 template <typename OutT>
