@@ -81,7 +81,8 @@ typedef struct swa_dims {
  *   k_cache, v_cache  [B][Hkv][W][d] bf16, updated in place
  *   k, v              [B][max_tokens][Hkv][d] bf16: row t of sequence b is the
  *                     token at position start_pos[b] + t
- *   max_tokens        row capacity of k / v, 1 <= max_tokens <= W
+ *   max_tokens        row capacity of k / v, 1 <= max_tokens <= W, and
+ *                     max_tokens * Hkv * d / 8 < 2^31 (else SWA_ERR_UNSUPPORTED)
  *   start_pos         device int32[B], >= 0
  *   n_tokens          device int32[B], 0 <= n_tokens[b] <= max_tokens: rows
  *                     [0, n_tokens[b]) are written, the rest ignored
