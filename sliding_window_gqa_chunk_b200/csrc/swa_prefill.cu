@@ -6,7 +6,7 @@
 // share a kv head (GQA: both heads reuse every K/V tile the CTA loads) of one
 // sequence.  With a workspace the grid is one CTA per SM and each CTA takes
 // units, heaviest first, from a counter in the workspace; the units of the
-// last round are cut into pieces of their key range whose partial softmax
+// last wave are cut into pieces of their key range whose partial softmax
 // results are merged by log-sum-exp.  Without one, the grid has one CTA per
 // unit.  Warp roles:
 //   warps 0-3  softmax for head slot 0 (TMEM lanes 0-127 = the 128 query rows)
@@ -1145,7 +1145,7 @@ PrefillSchedule prefill_schedule(long long n_units, int n_wtiles, int n_sms, boo
   if (!have_workspace || n_units < 1) return sc;
   long long ctas = n_sms < kMaxPersistentCtas ? n_sms : kMaxPersistentCtas;
   if (ctas < 1) ctas = 1;
-  // Units are taken heaviest first, so the last round over the SMs is the one
+  // Units are taken heaviest first, so the last wave over the SMs is the one
   // that can leave SMs idle (with fewer units than SMs, the only round).  Its
   // units (the last `tail` in the order) are cut into pieces of their key
   // range so that the round fills the SMs: at most ctas pieces in all, at most

@@ -144,7 +144,7 @@ def test_prefill_matches_oracle(B, lengths, W, chunk, Hq, Hkv, d, workspace):
 
 # Shapes with few units per call, so the persistent schedule cuts every unit
 # that sees at least 8 key tiles into 2-4 pieces of its key range and merges
-# them (the path a 4096-token chunk takes for its last round of units).
+# them (the path a 4096-token chunk takes for its last wave of units).
 SPLIT_CASES = [
     # B, lengths,      W,    chunk, Hq, Hkv, d
     (1, [2304],        2048, 256,   4,  2,   128),   # 4 units per call: 4 pieces each
