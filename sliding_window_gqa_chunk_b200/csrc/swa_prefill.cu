@@ -1146,7 +1146,7 @@ PrefillSchedule prefill_schedule(long long n_units, int n_wtiles, int n_sms, boo
   long long ctas = n_sms < kMaxPersistentCtas ? n_sms : kMaxPersistentCtas;
   if (ctas < 1) ctas = 1;
   // Units are taken heaviest first, so the last wave over the SMs is the one
-  // that can leave SMs idle (with fewer units than SMs, the only round).  Its
+  // that can leave SMs idle (with fewer units than SMs, the only wave).  Its
   // units (the last `tail` in the order) are cut into pieces of their key
   // range so that the round fills the SMs: at most ctas pieces in all, at most
   // 4 per unit, about 4 or more key tiles each for a unit that sees a whole
