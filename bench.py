@@ -49,8 +49,8 @@ METRIC = ("prefill tokens/s & TFLOP/s (% bf16 peak); decode tokens/s & HBM GB/s 
 # while the kernel source is the one that was profiled (sha256 prefix of the .cu file);
 # the summaries with the commands are under profiles/.
 PROFILED_TRAFFIC = {
-    "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "27462eefd1af7929",
-                           "bytes": 67_757_312 + 15_459_584,
+    "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "dcf56dfe57ae65f1",
+                           "bytes": 67_441_920 + 14_799_872,
                            "launch": "chunk 1 of 4 (every row sees 4096 keys)"},
     "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "162841c6a1d30b0e",
                           "bytes": 1_074_293_248 + 3_966_976, "launch": "one decode step"},
