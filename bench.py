@@ -52,8 +52,8 @@ PROFILED_TRAFFIC = {
     "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "dcf56dfe57ae65f1",
                            "bytes": 67_441_920 + 14_799_872,
                            "launch": "chunk 1 of 4 (every row sees 4096 keys)"},
-    "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "162841c6a1d30b0e",
-                          "bytes": 1_074_293_248 + 3_966_976, "launch": "one decode step"},
+    "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "525cf5410e872618",
+                          "bytes": 1_074_341_120 + 3_614_464, "launch": "one decode step"},
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
