@@ -46,13 +46,13 @@ from swa_workloads import (DECODE_B64, PREFILL_16K, decode_32l_workload, decode_
 METRIC = ("prefill tokens/s & TFLOP/s (% bf16 peak); decode tokens/s & HBM GB/s (% peak)")
 
 # DRAM bytes (read + write) per launch from one ncu capture of each kernel, valid only
-# while the kernel source is the one that was profiled (sha256 prefix of the .cu file);
-# the summaries with the commands are under profiles/.
+# while the kernel source is the one that was profiled (source_key: sha256 prefix of the
+# .cu file without comments); the summaries with the commands are under profiles/.
 PROFILED_TRAFFIC = {
-    "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "dcf56dfe57ae65f1",
+    "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "5afc8766efa7e304",
                            "bytes": 67_441_920 + 14_799_872,
                            "launch": "chunk 1 of 4 (every row sees 4096 keys)"},
-    "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "525cf5410e872618",
+    "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "c8020a7589bbd304",
                           "bytes": 1_074_341_120 + 3_614_464, "launch": "one decode step"},
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -199,16 +199,27 @@ def reduce_max(x: float, world: int) -> float:
     return float(t.item())
 
 
+def source_key(path: str) -> str:
+    """sha256 prefix of a CUDA source with its comments and blank space removed,
+    so that an edit of comments alone keeps a profile's record valid."""
+    import hashlib
+    import re
+    text = open(path, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)   # block comments
+    text = re.sub(r"//[^\n]*", " ", text)                 # line comments
+    text = " ".join(text.split())
+    return hashlib.sha256(text.encode()).hexdigest()[:16]
+
+
 def profiled_traffic(kernel: str):
     """ncu DRAM bytes per launch if the kernel source still matches the profiled one."""
-    import hashlib
     rec = PROFILED_TRAFFIC[kernel]
     path = os.path.join(ROOT, "sliding_window_gqa_chunk_b200", "csrc", rec["file"])
     try:
-        sha = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+        key = source_key(path)
     except OSError:
         return None, None
-    if sha != rec["sha"]:
+    if key != rec["sha"]:
         return None, None
     return rec["bytes"], rec["launch"]
 

@@ -13,13 +13,16 @@
 //   S^T[slot][head] = K[slot][:] . Q[head][:]    (M = 16 slots, N = 8 heads, K = d)
 //   O^T[d][head]   += V^T[d][slot] . P^T[slot][head]  (M = 16 d, N = 8 heads, K = 16 slots)
 //
-// Fragments come straight from global memory with 16-byte loads, no shared
-// memory: a dot product over d is invariant under any permutation of d applied
-// to both K and Q, so each lane loads contiguous 16-byte pieces and the d index
-// is relabelled to match the mma fragment layout; the PV product uses a second
-// relabelling of d (undone when O is stored) and pairs consecutive slots with
-// byte permutes.  P^T goes from the S accumulator layout to the B-operand
-// layout with one movmatrix.trans per 8x8 block.
+// Each lane loads contiguous 16-byte pieces of K and V rows: a dot product
+// over d is invariant under any permutation of d applied to both K and Q, so
+// the d index is relabelled to match the mma fragment layout; the PV product
+// uses a second relabelling of d (undone when O is stored) and pairs
+// consecutive slots with byte permutes.  P^T goes from the S accumulator
+// layout to the B-operand layout with one movmatrix.trans per 8x8 block.
+// With at least one (sequence, kv head) pair per SM the pieces come straight
+// from global memory (register-fed variant); with fewer pairs a producer warp
+// streams each split into a shared-memory ring with bulk copies and the
+// compute warps read their pieces from there (stream variant).
 //
 // Work split: grid (n_splits, Hkv, B); a CTA of NW warps covers one split of
 // the W slots; warps take interleaved 16-slot blocks and merge their (m, l, O)
