@@ -92,6 +92,22 @@ def test_profiled_traffic_is_dropped_when_the_kernel_changes(monkeypatch):
     assert bench.profiled_traffic("swa_decode_kernel") == (None, None)
 
 
+def test_profiled_traffic_matches_the_current_sources():
+    for kernel in ("swa_prefill_kernel", "swa_decode_kernel"):
+        assert bench.profiled_traffic(kernel)[0] is not None, f"{kernel}: profile record is stale"
+
+
+def test_source_key_ignores_comments_but_not_code(tmp_path):
+    base = "__global__ void k(int* p) {\n  p[0] = 1;  // one\n}\n"
+    f = tmp_path / "a.cu"
+    f.write_text(base)
+    key = bench.source_key(str(f))
+    f.write_text("/* header */\n" + base.replace("// one", "// the first element"))
+    assert bench.source_key(str(f)) == key
+    f.write_text(base.replace("p[0] = 1", "p[0] = 2"))
+    assert bench.source_key(str(f)) != key
+
+
 def test_decode_launch_count_follows_the_split_rule():
     import sliding_window_gqa_chunk_b200 as swa
     mk = lambda B: swa.Dims(B, 32, 8, 128, 4096, 1.0 / 128 ** 0.5, "bf16")
