@@ -236,6 +236,57 @@ def test_prefill_chunk_after_decode_steps():
     swa.device_status()
 
 
+def test_prefill_chunks_replayed_from_a_cuda_graph():
+    """The prefill and append kernels are launched with programmatic dependent
+    launch: a CUDA graph of a whole prompt (chunk, append, chunk, append, ...)
+    replayed twice gives the eager result bit for bit, and the oracle's."""
+    B, L, W, Hq, Hkv, d = 2, 768, 256, 8, 2, 128
+    q, k, v = random_case(909, B, L, Hq, Hkv, d)
+    dims = mk_dims(B, Hq, Hkv, d, W)
+    n = L // W
+    qs = [q[:, c * W:(c + 1) * W].contiguous().to(DEV) for c in range(n)]
+    ks = [k[:, c * W:(c + 1) * W].contiguous().to(DEV) for c in range(n)]
+    vs = [v[:, c * W:(c + 1) * W].contiguous().to(DEV) for c in range(n)]
+    sps = [dev_i32([c * W] * B) for c in range(n)]
+    nt = dev_i32([W] * B)
+    ws = swa.prefill_workspace(dims, W, DEV)
+
+    def prompt(kc, vc, outs):
+        for c in range(n):
+            swa.prefill_chunk(dims, outs[c], qs[c], ks[c], vs[c], kc, vc, sps[c], nt, workspace=ws)
+            swa.cache_append(dims, kc, vc, ks[c], vs[c], sps[c], nt)
+
+    kc_e, vc_e = swa.new_cache(dims, DEV)
+    outs_e = [torch.zeros((B, W, Hq, d), dtype=torch.float32, device=DEV) for _ in range(n)]
+    prompt(kc_e, vc_e, outs_e)
+    torch.cuda.synchronize()
+    swa.device_status()
+
+    kc_g, vc_g = swa.new_cache(dims, DEV)
+    outs_g = [torch.full((B, W, Hq, d), float("nan"), dtype=torch.float32, device=DEV) for _ in range(n)]
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            prompt(kc_g, vc_g, outs_g)
+    torch.cuda.current_stream().wait_stream(side)
+    for _ in range(2):
+        kc_g.zero_()
+        vc_g.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        swa.device_status()
+        for c in range(n):
+            assert torch.equal(outs_g[c], outs_e[c]), f"chunk {c}"
+        assert torch.equal(kc_g, kc_e) and torch.equal(vc_g, vc_e)
+    ref, rcache = oracle.run_chunked_prefill(q, k, v, W, W, dims.scale)
+    got = torch.cat([o.double().cpu() for o in outs_g], dim=1).numpy()
+    assert_close(got, ref, "prefill from a CUDA graph")
+    np.testing.assert_array_equal(cache_as_f64(kc_g), rcache.k)
+    del graph
+
+
 # ----------------------------------------------------------------------------
 # Decode against the oracle
 # ----------------------------------------------------------------------------
