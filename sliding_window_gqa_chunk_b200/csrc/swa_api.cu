@@ -155,20 +155,26 @@ int encode_map(EncodeTiledFn fn, CUtensorMap* map, const void* ptr, int rank, co
   return SWA_OK;
 }
 
-// The five TMA descriptors of a prefill call depend only on the tensors'
+// The TMA descriptors of a prefill call depend only on the tensors'
 // addresses and the shape, so they are kept for repeated calls (a prompt's
 // chunks, a decode loop that feeds one-token chunks): a small cache, replaced
 // round robin, keyed by device, pointers and shape.
 struct MapKey {
   int device;
-  const void* ptr[5];
-  int batch, n_q_heads, n_kv_heads, head_dim, window, max_tokens;
+  const void* ptr[6];
+  int batch, n_q_heads, n_kv_heads, head_dim, window, max_tokens, out_dtype;
   bool operator==(const MapKey& o) const {
     return device == o.device && memcmp(ptr, o.ptr, sizeof(ptr)) == 0 && batch == o.batch &&
            n_q_heads == o.n_q_heads && n_kv_heads == o.n_kv_heads && head_dim == o.head_dim &&
-           window == o.window && max_tokens == o.max_tokens;
+           window == o.window && max_tokens == o.max_tokens && out_dtype == o.out_dtype;
   }
 };
+
+// Whole output tiles of the prefill go out through shared memory and a TMA
+// store for bf16 output at d = 128 (the kernel has the staging buffer there).
+bool prefill_out_tma(const swa_dims* dims) {
+  return dims->out_dtype == SWA_DTYPE_BF16 && dims->head_dim == 128;
+}
 constexpr int kMapCacheSize = 16;
 std::mutex g_map_mu;
 MapKey g_map_keys[kMapCacheSize];
@@ -184,7 +190,8 @@ extern "C" SWA_API void swa_debug_fail_encode(int on) { g_fail_encode = on; }
 #endif
 
 int prefill_maps(int device, const swa_dims* dims, int max_tokens, const void* q, const void* k,
-                 const void* v, const void* k_cache, const void* v_cache, swa::PrefillMaps* out) {
+                 const void* v, const void* k_cache, const void* v_cache, const void* o,
+                 swa::PrefillMaps* out) {
 #ifdef SWA_TEST_FAULTS
   if (g_fail_encode)
     return fail(SWA_ERR_CUDA, "cuTensorMapEncodeTiled(q) failed with CUresult %d (injected)",
@@ -198,6 +205,8 @@ int prefill_maps(int device, const swa_dims* dims, int max_tokens, const void* q
   key.ptr[2] = v;
   key.ptr[3] = k_cache;
   key.ptr[4] = v_cache;
+  key.ptr[5] = o;
+  key.out_dtype = dims->out_dtype;
   key.batch = dims->batch;
   key.n_q_heads = dims->n_q_heads;
   key.n_kv_heads = dims->n_kv_heads;
@@ -227,6 +236,9 @@ int prefill_maps(int device, const swa_dims* dims, int max_tokens, const void* q
     cuuint64_t str4[3] = {D * es, (cuuint64_t)Hq * D * es, (cuuint64_t)max_tokens * Hq * D * es};
     cuuint32_t box4[4] = {(cuuint32_t)box_d, 1, 128, 1};
     if ((rc = encode_map(enc, &maps.q, q, 4, dims4, str4, box4, swz, "q"))) return rc;
+    // the output has the shape and element type of q
+    if (prefill_out_tma(dims) && (rc = encode_map(enc, &maps.out, o, 4, dims4, str4, box4, swz, "out")))
+      return rc;
   }
   {
     cuuint64_t dims4[4] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)max_tokens, (cuuint64_t)B};
@@ -433,7 +445,7 @@ int swa_prefill_chunk(const swa_dims* dims, void* out, const void* q, const void
   cudaError_t e = cudaGetDevice(&device);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   swa::PrefillMaps maps;
-  if ((rc = prefill_maps(device, dims, max_tokens, q, k, v, k_cache, v_cache, &maps))) return rc;
+  if ((rc = prefill_maps(device, dims, max_tokens, q, k, v, k_cache, v_cache, out, &maps))) return rc;
 
   const swa::PrefillSchedule sc =
       swa::prefill_schedule(n_units, (W + 127) / 128, swa::device_sm_count(device), workspace != nullptr);
@@ -459,6 +471,7 @@ int swa_prefill_chunk(const swa_dims* dims, void* out, const void* q, const void
   p.out_f32 = dims->out_dtype == SWA_DTYPE_F32;
   // every row and 16-element piece of a row starts 32 bytes apart from the base
   p.out_v8 = (reinterpret_cast<uintptr_t>(out) % 32) == 0;
+  p.out_tma = prefill_out_tma(dims) ? 1 : 0;
   p.trace = g_trace;
   e = swa::launch_prefill(p, maps, (int)sc.grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "swa_prefill_chunk launch");

@@ -80,6 +80,8 @@ struct PrefillParams {
   float scale_log2;
   int out_f32;
   int out_v8;                   // 1: out is 32-byte aligned (the epilogue stores 32 bytes per instruction)
+  int out_tma;                  // 1: whole output tiles go out through shared memory and a TMA
+                                // store (bf16 output, d = 128; maps.out is encoded)
   void* workspace;              // caller scratch (NULL: no key-range splits)
   int* trace;                   // progress words in host-mapped memory (trace builds only)
 };
@@ -98,6 +100,7 @@ struct PrefillMaps {
   CUtensorMap v;
   CUtensorMap kc;       // k_cache [B*Hkv][W][d] box {d_box, 128, 1}
   CUtensorMap vc;
+  CUtensorMap out;      // out [B][T][Hq][d] bf16, box {d_box, 1, 128, 1} (out_tma only)
 };
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);

@@ -116,7 +116,7 @@ static_assert(kWsMergeOffset + kMaxPersistentCtas * 8 * sizeof(int) <= kWsPartia
 
 // K / V ring depths for head_dim 128 (2 Q tiles + K + V must fit in 227 KB).
 #ifndef SWA_K_STAGES_D128
-#define SWA_K_STAGES_D128 3
+#define SWA_K_STAGES_D128 2
 #endif
 #ifndef SWA_V_STAGES_D128
 #define SWA_V_STAGES_D128 2
@@ -136,7 +136,10 @@ struct Cfg {
   static constexpr uint32_t kLayout = (kSwzBytes == 128) ? tc::kLayoutSW128 : tc::kLayoutSW32;
   static constexpr int kSBO = 8 * kSwzBytes;                       // stride of 8-row groups
   static constexpr int kKStepsPerBlock = kSwzBytes / 32;           // 16-element k-steps per box row
-  static constexpr int kSmemTiles = (2 + kKStages + kVStages) * kTileBytes;
+  // d = 128: one 128 x d bf16 tile of shared memory stages a head's output
+  // for a TMA store (the two head slots take turns)
+  static constexpr int kStageBytes = (D == 128) ? kTileBytes : 0;
+  static constexpr int kSmemTiles = (2 + kKStages + kVStages) * kTileBytes + kStageBytes;
   static constexpr int kSmemBytes = kSmemTiles + 512 + 1024;       // barriers + alignment slack
   static_assert(kColBlocks * kSwzBytes == D * 2, "head_dim must fill whole swizzle rows");
 };
@@ -403,6 +406,7 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
   const uint32_t sQ = base;                                   // 2 tiles
   const uint32_t sK = base + 2 * C::kTileBytes;               // NK tiles
   const uint32_t sV = sK + NK * C::kTileBytes;                // NV tiles
+  const uint32_t sStage = sV + NV * C::kTileBytes;            // output staging tile (d = 128)
   const uint32_t sBar = base + C::kSmemTiles;
   // barrier addresses (8 bytes each)
   const uint32_t bar_q_full = sBar;
@@ -418,7 +422,9 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
   const uint32_t bar_item_empty = bar_item_full + 16;  // [2]
   const uint32_t bar_done = bar_item_empty + 16;
   const uint32_t bar_fetch = bar_done + 8;             // K producer done issuing an item
-  static_assert(16 + 16 * NK + 16 * NV + 5 * 16 + 16 <= 320, "barrier area");
+  const uint32_t bar_stage_free = bar_fetch + 8;       // the staging tile has been read by its TMA store
+  const uint32_t bar_stage_full = bar_stage_free + 8;  // [2] a head slot's rows are in the staging tile
+  static_assert(16 + 16 * NK + 16 * NV + 5 * 16 + 40 <= 320, "barrier area");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::kSmemTiles + 320);
   volatile int* item_rec = reinterpret_cast<volatile int*>(base_ptr + C::kSmemTiles + 336);  // [2][kRecInts]
   static_assert(336 + 2 * kRecInts * 4 <= 512, "item records must fit the control area");
@@ -446,6 +452,9 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
     }
     tc::mbar_init(bar_done, 1);
     tc::mbar_init(bar_fetch, 1);
+    tc::mbar_init(bar_stage_free, 1);
+    tc::mbar_init(bar_stage_full, kRows / 32);
+    tc::mbar_init(bar_stage_full + 8, kRows / 32);
     tc::mbar_fence_init();
   }
   if (threadIdx.x == 0) SWA_TRACE_AT(0, 1);
@@ -746,6 +755,8 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
     const float sl2 = p.scale_log2;
     int g0 = 0;   // S tiles before the current item
     int oi = 0;   // items with tiles (O barrier phase)
+    int n_staged = 0;  // items whose output went through the staging tile
+    bool stage_pending = false;  // this thread's TMA store may still be reading the staging tile
     bool ok = true;
     for (int it = 0; ok; ++it) {
       const volatile int* rec;
@@ -763,6 +774,12 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
       if (end) break;
       const int n_tiles = I.n_tiles;
       const int t = I.t_lo + row;               // chunk row
+      if (stage_pending) {
+        // the other head slot may use the staging tile once this store has read it
+        tc::bulk_wait_read_all();
+        tc::mbar_arrive(bar_stage_free);
+        stage_pending = false;
+      }
       const long long s = I.s;
       const long long pos_i = s + t;            // absolute query position
       // this row's visible cache slots: the cyclic range [a_i, a_i + len_i)
@@ -962,6 +979,48 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
         tc::tc_wait_ld();
 #pragma unroll
         for (int c = 0; c < D / 16; ++c) tc::reg_fence16(ov + c * 16);
+        if (C::kStageBytes > 0 && p.out_tma && I.t_lo + kRows <= I.n) {
+          // A whole tile of bf16 output: the head's rows go to the staging
+          // tile in the TMA box layout (128-byte swizzle: 16-byte chunk c of
+          // row r at (c ^ (r mod 8)) * 16), then one thread stores each column
+          // block with a TMA store.  The head slots take turns on the tile.
+          const int use = n_staged * hpc + i;
+          ++n_staged;
+          if (use > 0) {
+            ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_stage_free, (use - 1) & 1, p.status));
+            if (!ok) break;
+          }
+#pragma unroll
+          for (int cb = 0; cb < C::kColBlocks; ++cb) {
+#pragma unroll
+            for (int c = 0; c < C::kSwzBytes / 16; ++c) {
+              const float* v8 = ov + cb * C::kBoxD + c * 8;
+              tc::st_shared_v4(sStage + cb * C::kBlockBytes + row * C::kSwzBytes + ((c ^ (row & 7)) << 4),
+                               pack_bf16x2(v8[0] * inv_l, v8[1] * inv_l), pack_bf16x2(v8[2] * inv_l, v8[3] * inv_l),
+                               pack_bf16x2(v8[4] * inv_l, v8[5] * inv_l), pack_bf16x2(v8[6] * inv_l, v8[7] * inv_l));
+            }
+          }
+          // Each warp's writes reach the async proxy, then the warp counts
+          // itself; the head slot's first warp waits (bounded) for all four
+          // and issues the stores.
+          tc::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(bar_stage_full + 8 * i);
+          if ((warp & 3) == 0) {
+            ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_stage_full + 8 * i, (n_staged - 1) & 1, p.status));
+            if (!ok) break;
+            if (lane == 0) {
+#pragma unroll
+              for (int cb = 0; cb < C::kColBlocks; ++cb)
+                tc::tma_store_4d(&maps.out, cb * C::kBoxD, I.h_first + i, I.t_lo, I.b,
+                                 sStage + cb * C::kBlockBytes);
+              tc::bulk_commit_group();
+              stage_pending = true;  // released below, once the next item is under way
+            }
+            __syncwarp();
+          }
+          continue;
+        }
         if (t < I.n) {
 #pragma unroll
           for (int c = 0; c < D / 16; ++c)
@@ -1048,6 +1107,9 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
         if (t < I.n) store16<OutT>(dst + c * 16, ov, inv_l, p.out_v8 != 0);
       }
     }
+    // every TMA store of the output has completed before the CTA leaves
+    if ((warp & 3) == 0 && lane == 0) tc::bulk_wait_all();
+    if (stage_pending) tc::mbar_arrive(bar_stage_free);
     if (row == 0) SWA_TRACE_AT(3 + i, ok ? 8000 : 7500);
   }
   }
