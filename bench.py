@@ -49,8 +49,8 @@ METRIC = ("prefill tokens/s & TFLOP/s (% bf16 peak); decode tokens/s & HBM GB/s 
 # while the kernel source is the one that was profiled (source_key: sha256 prefix of the
 # .cu file without comments); the summaries with the commands are under profiles/.
 PROFILED_TRAFFIC = {
-    "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "25aa2c2cd0e8850c",
-                           "bytes": 67_442_432 + 16_320_768,
+    "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "9664eb26c2605ea5",
+                           "bytes": 67_821_312 + 14_862_080,
                            "launch": "chunk 1 of 4 (every row sees 4096 keys)"},
     "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "c8020a7589bbd304",
                           "bytes": 1_074_341_120 + 3_614_464, "launch": "one decode step"},

@@ -93,6 +93,10 @@ constexpr int kMmaWarp = 9;
 constexpr int kVProducerWarp = 10;
 constexpr int kFetchWarp = 11;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
+// A row's sum of p over one tile above which the optimistic exponentials are
+// redone against the tile's own max (2^32: far below fp32 overflow, so no p of
+// the optimistic pass can have overflowed unnoticed).
+constexpr float kOptimisticSumLimit = 4294967296.0f;
 constexpr uint32_t kTmemCols = 512;
 // Workspace layout: two scheduler counters; one merge counter per split unit
 // and softmax warp (at most one split unit per persistent CTA); then one fp32
@@ -848,22 +852,16 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
 
         // P = exp2(scale * log2(e) * s - base) for the whole tile, written over
         // the first 64 columns of S_i; returns this thread's sum of the fp32 p.
-        // With track_max it also returns the tile's largest raw score (the max
-        // chains run on the ALU pipe, beside the SFU exponentials).
-        auto exp_pass = [&](float base_neg, bool track_max, float& tile_max) -> float {
+        auto exp_pass = [&](float base_neg) -> float {
           const uint64_t sl2x2 = f2_pack(sl2, sl2);
           const uint64_t nbx2 = f2_pack(base_neg, base_neg);
           uint64_t lsum[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-          float m8[8];
-#pragma unroll
-          for (int a = 0; a < 8; ++a) m8[a] = -CUDART_INF_F;
 #pragma unroll
           for (int c = 0; c < kKeys / 32; ++c) {
             uint32_t pw[16];
 #pragma unroll
             for (int w = 0; w < 16; ++w) {
               const float s0 = sv[c * 32 + 2 * w], s1 = sv[c * 32 + 2 * w + 1];
-              if (track_max) m8[w % 8] = fmax3(m8[w % 8], s0, s1);
               const uint64_t x = f2_fma(f2_pack(s0, s1), sl2x2, nbx2);
               float p0, p1;
               f2_unpack(x, p0, p1);
@@ -878,8 +876,6 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
             }
             tc::tmem_st16(tS + c * 16, pw);  // P (bf16 pairs) over the first 64 columns of S_i
           }
-          if (track_max)
-            tile_max = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
           float a0, a1, b0, b1;
           f2_unpack(lsum[0], a0, a1);
           f2_unpack(lsum[1], b0, b1);
@@ -887,16 +883,18 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
         };
 
         // Optimistic pass: exponentiate against the running max right away and
-        // check the tile's max afterwards.  Only if some row's max grew by more
-        // than 2^8 (always on a row's first visible tile) is the tile redone
-        // against the new max.  The decisions are warp-uniform because the
-        // TMEM accesses they guard are warp-collective.
+        // look at the row's sum of p afterwards.  The running max may be stale
+        // (it moves only when a row's max grows by more than 2^8), so p can
+        // exceed 1; bf16 and fp32 keep their relative precision at any such
+        // scale.  A sum above 2^32, which any p above 2^32 (or an overflowed
+        // one) produces, sends the tile to the exact pass, as does a row's
+        // first visible tile.  The decisions are warp-uniform because the TMEM
+        // accesses they guard are warp-collective.
         float part = 0.f;
         bool exact = __any_sync(0xffffffffu, m_run == -CUDART_INF_F);
         if (!exact) {
-          float tmax;
-          part = exp_pass(-m_run, true, tmax);
-          exact = __any_sync(0xffffffffu, tmax * sl2 > m_run + kRescaleThreshold);
+          part = exp_pass(-m_run);
+          exact = __any_sync(0xffffffffu, !(part <= kOptimisticSumLimit));
         }
         if (exact) {
           // row maximum: 8 independent 3-input max chains, then a short tree
@@ -936,8 +934,7 @@ swa_prefill_kernel(const PrefillParams p, const __grid_constant__ PrefillMaps ma
               tc::tmem_st16(tO + c * 16, ow);
             }
           }
-          float unused;
-          part = exp_pass((m_run == -CUDART_INF_F) ? 0.f : -m_run, false, unused);
+          part = exp_pass((m_run == -CUDART_INF_F) ? 0.f : -m_run);
         }
         l_run += part;
         tc::tc_wait_st();
