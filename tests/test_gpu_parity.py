@@ -309,6 +309,12 @@ DECODE_CASES = [
     (3, 4096, 32, 8, 128, [4096, 12345, 700], 2),
     # 64 pairs: clusters of 2 (2048 slots each)
     (8, 4096, 32, 8, 128, [4096, 9000, 100, 4095, 20000, 7000, 1, 5000], 2),
+    # 8 pairs: clusters of 8 (512 slots per CTA); then a cache holding 101
+    # positions, so 7 of the 8 CTAs of each cluster see no slot
+    (1, 4096, 32, 8, 128, [40000], 3),
+    (1, 4096, 32, 8, 128, [100], 2),
+    # 4 pairs: clusters of 8, G = 4
+    (1, 4096, 16, 4, 128, [4096], 2),
 ]
 
 
