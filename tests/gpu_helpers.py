@@ -4,7 +4,9 @@ Python binding of the C ABI, and the tolerance check against the oracle.
 Tolerances (the same as the pass bar for attention outputs from bf16 inputs
 with fp32 accumulation): max |gpu - ref| <= 1e-2 and
 sum |gpu - ref| / sum |ref| <= 2e-3, with fp32 outputs.  bf16 outputs carry
-one more rounding (relative 2^-9) and are held to 1e-2 / 4e-3.
+one more rounding, of at most half a bf16 ulp of the value (2^-8 relative):
+they are held to 4e-3 in the sum, and each element to 1e-2 beyond that
+half ulp (an output near 4 alone can be off by 2^-7 after rounding).
 """
 import numpy as np
 import torch
@@ -37,8 +39,19 @@ def assert_close(got, ref, what="", bf16_out=False):
     rl = rel_l1(got, ref)
     bar = REL_L1_BF16_OUT if bf16_out else REL_L1
     MEASURED.append((what, mx, rl, bar))
-    assert mx <= MAX_ABS and rl <= bar, f"{what}: max_abs={mx:.3e} rel_l1={rl:.3e}"
+    excess = err
+    if bf16_out and err.size:
+        excess = err - bf16_half_ulp(ref)
+    mx_excess = float(excess.max()) if err.size else 0.0
+    assert mx_excess <= MAX_ABS and rl <= bar, f"{what}: max_abs={mx:.3e} rel_l1={rl:.3e}"
     return mx, rl
+
+
+def bf16_half_ulp(x):
+    """Half the spacing of bf16 numbers at |x| (8 significant bits)."""
+    a = np.maximum(np.abs(np.asarray(x, dtype=np.float64)), 2.0 ** -126)
+    _, e = np.frexp(a)  # a in [2^(e-1), 2^e)
+    return np.ldexp(1.0, e - 9)
 
 
 def dev_i32(values, device="cuda"):

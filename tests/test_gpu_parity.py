@@ -16,7 +16,8 @@ import torch
 import oracle
 import sliding_window_gqa_chunk_b200 as swa
 from swa_workloads import random_case, tiny_inputs, TINY_PREFILL, TINY_SHAPE
-from tests.gpu_helpers import (assert_close, cache_as_f64, dev_i32, gpu_chunked_prefill)
+from tests.gpu_helpers import (MEASURED, REL_L1, assert_close, cache_as_f64, dev_i32,
+                               gpu_chunked_prefill, rel_l1)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -163,6 +164,48 @@ def test_prefill_split_pieces_match_oracle(B, lengths, W, chunk, Hq, Hkv, d):
     ref, rcache = oracle.run_chunked_prefill(q, k, v, W, chunk, dims.scale, lengths=lengths)
     assert_close(got, ref, f"split pieces B={B} L={lengths} W={W} chunk={chunk}")
     np.testing.assert_array_equal(cache_as_f64(kc), rcache.k)
+
+
+# Score spikes: key kappa is set to alpha times the query of row r (first head of
+# its kv group), so that row's score for kappa exceeds everything it has seen by
+# about 16 * alpha in log2 units.  Spikes of 4 land far above the 2^32 bound of
+# the optimistic exponentials: the tile is redone against the new max, so the
+# spike's p is exactly 1.  Spikes of 1.5 stay below it: the row keeps its stale
+# max and the spike's p (about 2^19) is rounded to bf16 before the P V product
+# while the row sum holds it in fp32.  For a row that one key dominates, that
+# rounding moves the output by up to half a bf16 ulp of p relative, i.e.
+# 2^-8 |v| -- the same size as rounding the output itself to bf16.  Held to
+# that bound (plus 1e-3) element by element and to 2e-3 in the normalised L1.
+SPIKES = [  # (row, key, alpha)
+    (700, 600, 4.0), (900, 530, 4.0), (1000, 390, 4.0), (610, 230, 4.0),
+    (300, 200, 1.5), (1010, 140, 1.5), (820, 700, 1.5),
+]
+
+
+@pytest.mark.parametrize("workspace", [True, False], ids=["persistent", "grid"])
+def test_prefill_score_spikes_match_oracle(workspace):
+    B, L, W, chunk, Hq, Hkv, d = 1, 1024, 1024, 512, 4, 2, 128
+    q, k, v = random_case(4242, B, L, Hq, Hkv, d)
+    G = Hq // Hkv
+    for r, kappa, alpha in SPIKES:
+        assert kappa < r
+        for kvh in range(Hkv):
+            k[0, kappa, kvh] = (alpha * q[0, r, kvh * G].float()).to(torch.bfloat16)
+    dims = mk_dims(B, Hq, Hkv, d, W)
+    got, _, _ = gpu_chunked_prefill(dims, q, k, v, [L], chunk, workspace=workspace)
+    ref, _ = oracle.run_chunked_prefill(q, k, v, W, chunk, dims.scale)
+    what = f"score spikes ({'persistent' if workspace else 'grid'})"
+    err = np.abs(got - ref)
+    rl = rel_l1(got, ref)
+    vmax = float(v.abs().max())
+    MEASURED.append((what, float(err.max()), rl, REL_L1))
+    assert np.isfinite(got).all()
+    assert float(err.max()) <= 2.0 ** -8 * vmax + 1e-3, f"{what}: max_abs={err.max():.3e}"
+    assert rl <= REL_L1, f"{what}: rel_l1={rl:.3e}"
+    # the rows redone against their spike attend almost only to that key
+    for r, kappa, alpha in SPIKES:
+        if alpha >= 4.0:
+            np.testing.assert_allclose(got[0, r, 0], v[0, kappa, 0].double().numpy(), atol=1e-3)
 
 
 def test_prefill_bf16_output():
