@@ -26,6 +26,9 @@
 //   2^8), and write P_i = exp2(...) as bf16 back over S_i in TMEM
 //   O_i += P_i V_j        tcgen05.mma, A = P (TMEM), B = V (smem, d-contiguous)
 // Tensor memory: S_0 | S_1 | O_0 | O_1  (128 + 128 + d + d columns of 512).
+// The epilogue divides O_i by the row sum; whole 128-row tiles of bf16 output
+// at d = 128 leave through a shared-memory staging tile and TMA stores, other
+// rows are stored from registers.
 //
 // Key tiles: the keys of a chunk are the cache slots holding positions
 // [max(0, s + t_lo - W + 1), s) and the chunk rows [0, t_hi].  The cache
