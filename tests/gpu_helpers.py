@@ -17,9 +17,9 @@ MAX_ABS = 1e-2
 REL_L1 = 2e-3
 REL_L1_BF16_OUT = 4e-3
 
-# (what, max_abs, rel_l1, bar) of every comparison made in this session; the
-# conftest prints them at the end of the run so the measured errors are on
-# record next to the pass/fail verdict.
+# (what, max_abs, rel_l1, rel_l1 bar, max_abs bar as text) of every comparison
+# made in this session; the conftest prints them at the end of the run so the
+# measured errors are on record next to the pass/fail verdict.
 MEASURED = []
 
 
@@ -38,7 +38,7 @@ def assert_close(got, ref, what="", bf16_out=False):
     mx = float(err.max()) if err.size else 0.0
     rl = rel_l1(got, ref)
     bar = REL_L1_BF16_OUT if bf16_out else REL_L1
-    MEASURED.append((what, mx, rl, bar))
+    MEASURED.append((what, mx, rl, bar, "1e-2 + half ulp" if bf16_out else "1e-2"))
     excess = err
     if bf16_out and err.size:
         excess = err - bf16_half_ulp(ref)
