@@ -218,6 +218,31 @@ def test_prefill_bf16_output():
     assert_close(got, ref, "bf16 out", bf16_out=True)
 
 
+# bf16 output at d = 128: whole 128-row tiles leave through the shared-memory
+# staging tile and TMA stores, ragged tiles and merged split pieces from
+# registers.  One head per CTA (odd group sizes) and many units per persistent
+# CTA exercise the staging tile's hand-over between items.
+TMA_STORE_CASES = [
+    # B, lengths,                  W,    chunk, Hq, Hkv, workspace
+    (4, [2048, 2000, 1500, 777],   1024, 1024,  8,  8,  True),    # G = 1, up to 2 units per CTA
+    (4, [2048, 2000, 1500, 777],   1024, 1024,  8,  8,  False),   # the same, one CTA per unit
+    (2, [1100, 1300],              1024, 512,   6,  2,  True),    # G = 3, split pieces
+    (3, [640, 129, 1024],          256,  256,   8,  2,  True),    # G = 4, two heads per CTA
+]
+
+
+@pytest.mark.parametrize("B,lengths,W,chunk,Hq,Hkv,workspace", TMA_STORE_CASES)
+def test_prefill_bf16_output_staged_stores(B, lengths, W, chunk, Hq, Hkv, workspace):
+    d = 128
+    L = max(lengths)
+    q, k, v = random_case(5000 + W + chunk + Hq, B, L, Hq, Hkv, d, lengths=lengths)
+    dims = mk_dims(B, Hq, Hkv, d, W, out="bf16")
+    got, _, _ = gpu_chunked_prefill(dims, q, k, v, lengths, chunk, workspace=workspace)
+    ref, _ = oracle.run_chunked_prefill(q, k, v, W, chunk, dims.scale, lengths=lengths)
+    assert_close(got, ref, f"bf16 staged stores B={B} L={lengths} W={W} chunk={chunk} G={Hq // Hkv}",
+                 bf16_out=True)
+
+
 @pytest.mark.parametrize("out_dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("d", [64, 128])
 def test_prefill_output_16_byte_aligned(out_dtype, d):
