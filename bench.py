@@ -52,8 +52,8 @@ PROFILED_TRAFFIC = {
     "swa_prefill_kernel": {"file": "swa_prefill.cu", "sha": "9664eb26c2605ea5",
                            "bytes": 67_821_312 + 14_862_080,
                            "launch": "chunk 1 of 4 (every row sees 4096 keys)"},
-    "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "c8020a7589bbd304",
-                          "bytes": 1_074_341_120 + 3_614_464, "launch": "one decode step"},
+    "swa_decode_kernel": {"file": "swa_decode.cu", "sha": "9924a131379beebb",
+                          "bytes": 1_074_292_992 + 3_978_496, "launch": "one decode step"},
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20

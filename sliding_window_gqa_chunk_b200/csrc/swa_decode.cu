@@ -197,6 +197,11 @@ constexpr int stream_ring_bytes() { return kStreamStages * 2 * kChunkSlots * D *
 // could skip a fill of a stage and take a later fill's parity for an earlier
 // one.  12 warps: chunks 3 apart, 2 stages per warp.
 constexpr int kStreamWarps = 12;
+// Groups of 9-16 query heads carry two n-tiles of accumulators per warp: 4
+// compute warps (5 in all, up to 255 registers a thread, no spills).  With 12
+// (at most 128 registers) the spills made a G = 16 step 25-30 % slower, with 8
+// (168 registers) 2-4 %.
+constexpr int kStreamWarpsWide = 4;
 
 // Row stride (floats) of the per-warp O partials in shared memory: one float
 // of padding spreads the rows that a warp's lanes store at once over the banks
@@ -657,7 +662,7 @@ cudaError_t launch_decode_d(const DecodeParams& p, cudaStream_t stream) {
   const int G = p.n_q_heads / p.n_kv_heads;
   if (p.stream) {
     if (G <= 8) return launch_decode_t<D, 1, kStreamWarps, OutT, true>(p, stream);
-    return launch_decode_t<D, 2, kStreamWarps, OutT, true>(p, stream);
+    return launch_decode_t<D, 2, kStreamWarpsWide, OutT, true>(p, stream);
   }
   if (G <= 8) return launch_decode_t<D, 1, 4, OutT, false>(p, stream);
   return launch_decode_t<D, 2, 4, OutT, false>(p, stream);

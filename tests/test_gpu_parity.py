@@ -384,6 +384,8 @@ DECODE_CASES = [
     (1, 4096, 32, 8, 128, [100], 2),
     # 4 pairs: clusters of 8, G = 4
     (1, 4096, 16, 4, 128, [4096], 2),
+    # G = 16 (two n-tiles of heads per warp) at d = 128: 8 pairs in clusters of 8
+    (4, 4096, 32, 2, 128, [9000, 4096, 100, 20000], 2),
 ]
 
 
