@@ -305,6 +305,52 @@ def test_prefill_chunk_after_decode_steps():
     swa.device_status()
 
 
+def test_positions_near_the_int32_limit():
+    """Positions are int32: a cache filled up to just below 2^31 - 1000, a chunk
+    there, then decode steps, all against the oracle (slot = position mod W
+    with positions near 2^31; no signed 32-bit overflow in any kernel)."""
+    B, W, Hq, Hkv, d = 2, 256, 4, 2, 128
+    S = [2 ** 31 - 1000, 2 ** 31 - 700]          # chunk starts
+    T, n = 200, [200, 150]
+    g = torch.Generator().manual_seed(31)
+    dims = mk_dims(B, Hq, Hkv, d, W)
+    kc, vc = swa.new_cache(dims, DEV)
+    ref = oracle.RollingCache(B, Hkv, W, d)
+    # the W positions before each chunk, appended in one call
+    kf = torch.randn(B, W, Hkv, d, generator=g).to(torch.bfloat16)
+    vf = torch.randn(B, W, Hkv, d, generator=g).to(torch.bfloat16)
+    starts = [s - W for s in S]
+    swa.cache_append(dims, kc, vc, kf.to(DEV), vf.to(DEV), dev_i32(starts), dev_i32([W] * B))
+    oracle.cache_append(ref, kf, vf, starts, [W] * B)
+    q = torch.randn(B, T, Hq, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, T, Hkv, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, T, Hkv, d, generator=g).to(torch.bfloat16)
+    o = torch.zeros((B, T, Hq, d), dtype=torch.float32, device=DEV)
+    sp, nt = dev_i32(S), dev_i32(n)
+    swa.prefill_chunk(dims, o, q.to(DEV), k.to(DEV), v.to(DEV), kc, vc, sp, nt,
+                      workspace=swa.prefill_workspace(dims, T, DEV))
+    swa.cache_append(dims, kc, vc, k.to(DEV), v.to(DEV), sp, nt)
+    expect = oracle.prefill_chunk(ref, q, k, v, S, n, dims.scale)
+    oracle.cache_append(ref, k, v, S, n)
+    got = o.double().cpu().numpy()
+    for b in range(B):   # rows past n_tokens are not written
+        assert_close(got[b, : n[b]], expect[b, : n[b]], f"chunk near 2^31, sequence {b}")
+    np.testing.assert_array_equal(cache_as_f64(kc), ref.k)
+    ws = swa.decode_workspace(dims, DEV)
+    for step in range(3):
+        pos = [s + m + step for s, m in zip(S, n)]
+        qd = torch.randn(B, Hq, d, generator=g).to(torch.bfloat16)
+        kd = torch.randn(B, Hkv, d, generator=g).to(torch.bfloat16)
+        vd = torch.randn(B, Hkv, d, generator=g).to(torch.bfloat16)
+        od = torch.zeros((B, Hq, d), dtype=torch.float32, device=DEV)
+        swa.decode(dims, od, qd.to(DEV), kd.to(DEV), vd.to(DEV), kc, vc, dev_i32(pos), ws)
+        expect = oracle.decode(ref, qd, kd, vd, pos, dims.scale)
+        assert_close(od.double().cpu().numpy(), expect, f"decode near 2^31, step {step}")
+    np.testing.assert_array_equal(cache_as_f64(kc), ref.k)
+    np.testing.assert_array_equal(cache_as_f64(vc), ref.v)
+    swa.device_status()
+
+
 def test_prefill_chunks_replayed_from_a_cuda_graph():
     """The prefill and append kernels are launched with programmatic dependent
     launch: a CUDA graph of a whole prompt (chunk, append, chunk, append, ...)
